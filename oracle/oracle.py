@@ -1,0 +1,145 @@
+"""Python front of the fp64 CPU oracle (``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the cpu_baseline / reference leg of ``bench.py`` may import this module.  The
+CUDA library never calls it and shares no code with it; the two meet only in
+the seeded inputs of ``shared_kv_caches_b200.workloads``.
+
+``build()`` compiles ``oracle.c`` with gcc into ``liboracle.so`` next to it.
+``decode()`` runs the oracle on a workload dict, ``decode_f64()`` on float64
+arrays (used by the pins that need inputs bf16 cannot hold), ``merge()`` is the
+split combine.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+VARIANT_IDS = {"gqa": 0, "mqa": 1, "mla": 2, "gla": 3, "mlra": 4}
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "variant", "batch", "num_q_heads", "num_kv", "d_nope", "d_rope",
+        "page_size", "max_pages_per_seq", "num_pages", "paged")]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (plain C, -O2, no fast-math) if it is missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread",
+                               "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        vp, i32p, dp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)
+        lib.orc_decode.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int32, vp, vp, vp, i32p, i32p,
+                                   ctypes.c_double, i32p, ctypes.c_int32, dp, dp, ctypes.c_int32]
+        lib.orc_decode.restype = ctypes.c_int
+        lib.orc_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, dp, dp, dp, dp]
+        lib.orc_merge.restype = None
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _ptr(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pages_per_seq,
+         num_pages, paged, elem_type, q_nope, q_rope, kv, block_table, seq_lens, sm_scale,
+         b_list, nthreads):
+    lib = _load()
+    shp = _Shape(VARIANT_IDS[variant], batch, num_q_heads, num_kv, d_nope, d_rope, page_size,
+                 max_pages_per_seq, num_pages, 1 if paged else 0)
+    dt = np.uint16 if elem_type == 0 else np.float64
+    q_nope = np.ascontiguousarray(q_nope, dtype=dt)
+    q_rope_arr = None if q_rope is None else np.ascontiguousarray(q_rope, dtype=dt)
+    kv = np.ascontiguousarray(kv, dtype=dt)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, dtype=np.int32)
+    if b_list is None:
+        b_list = np.arange(batch, dtype=np.int32)
+    b_list = np.ascontiguousarray(b_list, dtype=np.int32)
+    nb = len(b_list)
+    out = np.zeros((nb, num_q_heads, d_nope), dtype=np.float64)
+    lse_rows = num_q_heads * num_kv if variant == "mlra" else num_q_heads
+    lse = np.zeros((nb, lse_rows), dtype=np.float64)
+    rc = lib.orc_decode(ctypes.byref(shp), elem_type, q_nope.ctypes.data,
+                        None if q_rope_arr is None else q_rope_arr.ctypes.data, kv.ctypes.data,
+                        None if bt is None else _ptr(bt, ctypes.c_int32), _ptr(seq_lens, ctypes.c_int32),
+                        float(sm_scale), _ptr(b_list, ctypes.c_int32), nb,
+                        _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                        int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with status {rc}")
+    if variant == "mlra":
+        lse = lse.reshape(nb, num_q_heads, num_kv)
+    return out, lse
+
+
+def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None):
+    """fp64 decode attention of a workload dict (from ``workloads.make_inputs``).
+
+    Returns ``(out, lse)``: out ``[n_b][H][d_nope]`` float64 (MLRA: the sum
+    over branches), lse ``[n_b][H]`` (MLRA ``[n_b][H][R]``), natural log.
+    """
+    s = inputs["shape"]
+    scale = inputs["sm_scale"] if sm_scale is None else sm_scale
+    return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
+                inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 0,
+                inputs["q_nope"], inputs["q_rope"], inputs["kv"], inputs["block_table"],
+                inputs["seq_lens"], scale, b_list, nthreads)
+
+
+def decode_f64(variant, num_kv, q_nope, q_rope, kv, seq_lens, sm_scale, block_table=None,
+               page_size=64, b_list=None, nthreads=None):
+    """Same computation on float64 arrays in the same layouts.
+
+    ``q_nope`` is ``[B][H][d_nope]`` (MLRA ``[B][H][R][d_nope]``), ``kv`` is the
+    pool; without ``block_table`` the pool is contiguous per sequence.
+    """
+    q_nope = np.asarray(q_nope, dtype=np.float64)
+    batch, H = q_nope.shape[0], q_nope.shape[1]
+    d_nope = q_nope.shape[-1]
+    d_rope = 0 if q_rope is None else np.asarray(q_rope).shape[-1]
+    kv = np.asarray(kv, dtype=np.float64)
+    num_pages = kv.shape[0]
+    if block_table is None:
+        mpps = num_pages // batch
+    else:
+        mpps = np.asarray(block_table).shape[1]
+    return _run(variant, batch, H, num_kv, d_nope, d_rope, page_size, mpps, num_pages,
+                block_table is not None, 1, q_nope, q_rope, kv, block_table, seq_lens, sm_scale,
+                b_list, nthreads)
+
+
+def merge(o_s: np.ndarray, lse_s: np.ndarray):
+    """Combine per-part results: ``o_s [P][rows][dv]``, ``lse_s [P][rows]``."""
+    lib = _load()
+    o_s = np.ascontiguousarray(o_s, dtype=np.float64)
+    lse_s = np.ascontiguousarray(lse_s, dtype=np.float64)
+    P, rows, dv = o_s.shape
+    o = np.zeros((rows, dv), dtype=np.float64)
+    lse = np.zeros(rows, dtype=np.float64)
+    lib.orc_merge(P, rows, dv, _ptr(o_s, ctypes.c_double), _ptr(lse_s, ctypes.c_double),
+                  _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    return o, lse
