@@ -1,0 +1,181 @@
+/*
+ * kvattn.h -- C ABI of the B200 decode-attention library (libkvattn.so).
+ *
+ * One call computes single-token (decode) attention for a batch of sequences
+ * over a compressed or shared KV cache held in HBM:
+ *
+ *   out[b,h] = sum_j softmax_j( sm_scale * q[b,h] . k_j ) v_j     (j < seq_lens[b])
+ *
+ * MLA explainer (mlqm.cn/news/371735), section 2.3 gives the formula, section
+ * 2.2 the concatenations q = [q^C ; q^R], k = [k^C ; k^R] and that values are
+ * the latent part only; the MLRA page (aitntnews.com newId=23265) gives the
+ * absorbed decode form (MLA paragraph: W_UK absorbed into the query, decode
+ * becomes one 576-wide MQA head), the GQA and MQA bullets, the block
+ * decomposition and "moving the sum outside" (per-branch attention, branch
+ * outputs summed afterwards); the GLA page (jsbsmhs.com/zixun/902167, "Grouped
+ * Latent Attention") gives latent heads that each serve one group of query
+ * heads.  The MFA page (jsqmd.com/news/79551, "technical breakthrough") gives
+ * a single wide KV head, which decodes as MQA.
+ *
+ * Variants and what a unit of the cache is:
+ *   KVATTN_GQA  num_kv KV heads, query head h uses KV head h / (H / num_kv)
+ *   KVATTN_MQA  the same with num_kv = 1 (MFA at decode time: one wide head)
+ *   KVATTN_MLA  absorbed MLA: key = [latent (d_nope) ; rope key (d_rope)],
+ *               value = latent; num_kv = 1
+ *   KVATTN_GLA  num_kv = G latent heads of d_nope each plus one shared rope
+ *               key; head h uses latent h / (H / G)
+ *   KVATTN_MLRA num_kv = R branches of d_nope each plus one shared rope key;
+ *               every head attends every branch with its own query slice and
+ *               the R normalised branch outputs are summed (latent space)
+ *
+ * Memory (all device pointers, row-major, caller-owned):
+ *   q_nope     bf16 [B][H][d_nope]           (MLRA [B][H][R][d_nope])
+ *   q_rope     bf16 [B][H][d_rope]           (MLRA [B][H][R][d_rope]); NULL when
+ *              d_rope == 0 (GQA/MQA)
+ *   kv_cache   latent variants: bf16 [num_pages][page_size][num_kv*d_nope + d_rope],
+ *              each token row [c_0 | ... | c_{num_kv-1} | k_rope];
+ *              GQA/MQA: bf16 [num_pages][2 (K, V)][page_size][num_kv][d_nope]
+ *   block_table int32 [B][max_pages_per_seq]: physical page of each logical
+ *              64-token page; NULL = contiguous cache, sequence b owns pages
+ *              b*max_pages_per_seq .. b*max_pages_per_seq + max_pages_per_seq-1
+ *   seq_lens   int32 [B], 0 <= seq_lens[b] <= max_seq_len (read on the device)
+ *   out        [B][H][d_nope], bf16 (round to nearest even) or fp32
+ *   lse        fp32 [B][H] (MLRA [B][H][R]), natural log of the softmax
+ *              denominator including sm_scale; may be NULL
+ *   workspace  device scratch of kvattn_workspace_size() bytes, 256-byte
+ *              aligned, prepared once with kvattn_workspace_init()
+ *
+ * Token j of sequence b is slot j % 64 of page block_table[b][j / 64].
+ * Slots past seq_lens[b] may hold anything (NaN included) and never reach a
+ * result.  An empty sequence yields out = 0 and lse = -inf.
+ *
+ * Conventions: every call is asynchronous on `stream` (a cudaStream_t, NULL =
+ * legacy default stream) and returns a status before or after enqueueing;
+ * nothing is allocated per call and no host synchronisation happens except in
+ * kvattn_get_device_error().  Calls on different streams with different
+ * workspaces may run concurrently.  Bad arguments return a negative status
+ * without launching anything.  Bad data found on the device (a page id outside
+ * [0, num_pages), a sequence longer than max_seq_len) sets a bit in the
+ * workspace error word; the offending page is skipped, nothing traps.
+ */
+#ifndef KVATTN_H
+#define KVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum kvattn_variant {
+    KVATTN_GQA = 0,
+    KVATTN_MQA = 1,
+    KVATTN_MLA = 2,
+    KVATTN_GLA = 3,
+    KVATTN_MLRA = 4
+};
+
+enum kvattn_out_dtype { KVATTN_OUT_BF16 = 0, KVATTN_OUT_FP32 = 1 };
+
+enum kvattn_status {
+    KVATTN_OK = 0,
+    KVATTN_ERR_INVALID_ARG = -1,       /* null pointer, bad size, inconsistent shape */
+    KVATTN_ERR_UNSUPPORTED = -2,       /* valid request outside what the kernels cover */
+    KVATTN_ERR_WORKSPACE_TOO_SMALL = -3,
+    KVATTN_ERR_MISALIGNED = -4,        /* a pointer breaks the alignment rules below */
+    KVATTN_ERR_CUDA = -5               /* a CUDA launch or copy reported an error */
+};
+
+/* Bits of the device error word (kvattn_get_device_error). */
+enum kvattn_device_error {
+    KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1, /* block_table entry outside [0, num_pages): page skipped */
+    KVATTN_DEVERR_SEQ_TOO_LONG = 2,      /* seq_lens[b] > max_seq_len: clamped to max_seq_len */
+    KVATTN_DEVERR_WAIT_TIMEOUT = 4       /* a bounded wait on an mbarrier ran out: tile skipped */
+};
+
+/* Which decode kernel a plan uses. */
+enum kvattn_kernel {
+    KVATTN_KERNEL_GENERIC = 0,   /* CUDA-core split-KV kernel, any supported shape */
+    KVATTN_KERNEL_GQA = 1,       /* CUDA-core GQA/MQA kernel, bulk-copy staged pages */
+    KVATTN_KERNEL_LATENT_TC = 2, /* tcgen05/TMEM latent kernel (MLA, GLA, MLRA) */
+    KVATTN_KERNEL_MQA_TC = 3     /* tensor-core MQA kernel (one wide KV head) */
+};
+
+/*
+ * Problem description.  Alignment rules: q_nope, q_rope, kv_cache and out
+ * 16-byte aligned; lse 4-byte aligned; workspace 256-byte aligned.
+ * d_nope and d_rope must be multiples of 8; d_nope <= 512, d_rope <= 128.
+ * page_size must be 64.  max_seq_len is a host-side bound on seq_lens used to
+ * size the launch (no host read of device memory happens).  num_splits = 0
+ * lets the library choose how many parts each context is split into; a
+ * positive value forces it (clamped to the pages of the longest sequence).
+ */
+typedef struct {
+    int32_t batch;             /* B >= 1 */
+    int32_t num_q_heads;       /* H >= 1 */
+    int32_t num_kv;            /* KV heads (GQA/MQA), 1 (MLA), groups G (GLA), branches R (MLRA) */
+    int32_t d_nope;            /* head dim (GQA/MQA) or latent width per group/branch */
+    int32_t d_rope;            /* width of the shared rope key; 0 for GQA/MQA */
+    int32_t page_size;         /* 64 */
+    int32_t max_pages_per_seq; /* block_table row stride; capacity = max_pages_per_seq * 64 */
+    int32_t num_pages;         /* pages in the pool (bounds check of block_table) */
+    int32_t max_seq_len;       /* >= every seq_lens[b]; <= capacity */
+    int32_t num_splits;        /* 0 = library choice, > 0 forces */
+    int32_t out_dtype;         /* kvattn_out_dtype */
+} kvattn_params;
+
+/* What kvattn_decode will launch for a problem (host only, no CUDA calls). */
+typedef struct {
+    int32_t kernel;            /* kvattn_kernel */
+    int32_t num_splits;        /* parts per context */
+    int32_t pages_per_split;   /* 64-token pages per part */
+    int32_t ctas;              /* CTAs of the decode launch */
+    int32_t launches;          /* kernel launches per kvattn_decode call */
+    int32_t reserved;
+    uint64_t workspace_bytes;  /* required workspace */
+} kvattn_plan;
+
+/* Fill *plan for (variant, p).  Returns KVATTN_OK or INVALID_ARG/UNSUPPORTED.
+ * Host only; never touches the GPU. */
+int kvattn_get_plan(int32_t variant, const kvattn_params *p, kvattn_plan *plan);
+
+/* Bytes of workspace kvattn_decode needs for (variant, p): a 256-byte header
+ * holding the device error word, then the per-part lse [B][splits][rows] and
+ * normalised outputs [B][splits][rows][d_nope] in fp32 (rows = H, or H*R for
+ * MLRA).  Host only. */
+int kvattn_workspace_size(int32_t variant, const kvattn_params *p, size_t *bytes);
+
+/* Zero the workspace header (device error word) on `stream`.  Call once
+ * after allocating a workspace and after reading an error. */
+int kvattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode attention, enqueued on `stream`: a split-KV pass that writes one
+ * normalised partial output and lse per (sequence, head[, branch], part)
+ * into the workspace, then a combine pass that merges the parts by their
+ * lse (flash-decoding), sums the MLRA branches, places GLA group heads and
+ * casts to out_dtype.  Returns KVATTN_OK once enqueued, a negative status
+ * (nothing enqueued) for bad arguments, KVATTN_ERR_CUDA if a launch failed.
+ */
+int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
+                  const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
+                  float sm_scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/* Copy the device error word to *code (0 = none, else kvattn_device_error
+ * bits).  Synchronises `stream`.  Returns KVATTN_ERR_CUDA if the copy
+ * failed. */
+int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code);
+
+/* Static, human-readable name of a status code. */
+const char *kvattn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int kvattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVATTN_H */

@@ -64,8 +64,8 @@ typedef struct {
     const orc_shape *s;
     int elem_type;
     const void *q_nope, *q_rope, *kv;
-    const int32_t *block_table, *seq_lens, *b_list;
-    int32_t n_b;
+    const int32_t *block_table, *seq_lens, *b_list, *h_list;
+    int32_t n_b, n_h;
     double sm_scale;
     double *out, *lse;
     int32_t nthreads, tid;
@@ -191,11 +191,13 @@ static void *worker(void *arg)
         J->status = -2;
         goto done;
     }
-    size_t items = (size_t)J->n_b * H;
+    int nh = J->n_h;
+    size_t items = (size_t)J->n_b * nh;
     for (size_t it = (size_t)J->tid; it < items; it += (size_t)J->nthreads) {
-        int bi = (int)(it / H), h = (int)(it % H);
+        int bi = (int)(it / nh), hi = (int)(it % nh);
         int b = J->b_list[bi];
-        double *dst = J->out + ((size_t)bi * H + h) * dn;
+        int h = J->h_list ? J->h_list[hi] : hi;
+        double *dst = J->out + ((size_t)bi * nh + hi) * dn;
         if (s->variant == ORC_MLRA) {
             int R = s->num_kv;
             for (int d = 0; d < dn; ++d)
@@ -209,7 +211,7 @@ static void *worker(void *arg)
                 }
                 for (int d = 0; d < dn; ++d)
                     dst[d] += o[d];
-                J->lse[((size_t)bi * H + h) * R + r] = l;
+                J->lse[((size_t)bi * nh + hi) * R + r] = l;
             }
         } else {
             int u = 0;
@@ -220,7 +222,7 @@ static void *worker(void *arg)
                 J->status = -1;
                 goto done;
             }
-            J->lse[(size_t)bi * H + h] = l;
+            J->lse[(size_t)bi * nh + hi] = l;
         }
     }
 done:
@@ -232,16 +234,17 @@ done:
 }
 
 /*
- * Decode attention for the sequences listed in b_list (n_b of them).
+ * Decode attention for the sequences listed in b_list (n_b of them) and the
+ * heads listed in h_list (n_h of them; h_list = NULL means all H heads).
  * elem_type: 0 = inputs are bf16 bit patterns (uint16), 1 = inputs are double.
- * out: [n_b][H][d_nope] (MLRA: sum over branches); lse: [n_b][H] (MLRA
- * [n_b][H][R]).  Returns 0, -1 for a page id outside the pool, -2 when out of
- * memory, -3 for an invalid shape.
+ * out: [n_b][n_h][d_nope] (MLRA: sum over branches); lse: [n_b][n_h] (MLRA
+ * [n_b][n_h][R]).  Returns 0, -1 for a page id outside the pool, -2 when out
+ * of memory, -3 for an invalid shape.
  */
 int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const void *q_rope,
                const void *kv, const int32_t *block_table, const int32_t *seq_lens,
-               double sm_scale, const int32_t *b_list, int32_t n_b, double *out, double *lse,
-               int32_t nthreads)
+               double sm_scale, const int32_t *b_list, int32_t n_b, const int32_t *h_list,
+               int32_t n_h, double *out, double *lse, int32_t nthreads)
 {
     if (!s || s->variant < 0 || s->variant > 4 || s->num_kv <= 0 || s->num_q_heads <= 0 ||
         s->d_nope <= 0 || s->d_rope < 0 || s->page_size <= 0)
@@ -257,6 +260,11 @@ int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const 
         if (b < 0 || b >= s->batch || seq_lens[b] > s->max_pages_per_seq * s->page_size)
             return -3;
     }
+    if (!h_list)
+        n_h = s->num_q_heads;
+    for (int i = 0; h_list && i < n_h; ++i)
+        if (h_list[i] < 0 || h_list[i] >= s->num_q_heads)
+            return -3;
     if (nthreads < 1)
         nthreads = 1;
     orc_job *jobs = calloc((size_t)nthreads, sizeof(orc_job));
@@ -267,8 +275,8 @@ int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const 
         return -2;
     }
     for (int t = 0; t < nthreads; ++t) {
-        orc_job J = {s, elem_type, q_nope, q_rope, kv, block_table, seq_lens, b_list, n_b,
-                     sm_scale, out, lse, nthreads, t, 0};
+        orc_job J = {s, elem_type, q_nope, q_rope, kv, block_table, seq_lens, b_list, h_list,
+                     n_b, n_h, sm_scale, out, lse, nthreads, t, 0};
         jobs[t] = J;
     }
     int started = 0;

@@ -48,7 +48,8 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         vp, i32p, dp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)
         lib.orc_decode.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int32, vp, vp, vp, i32p, i32p,
-                                   ctypes.c_double, i32p, ctypes.c_int32, dp, dp, ctypes.c_int32]
+                                   ctypes.c_double, i32p, ctypes.c_int32, i32p, ctypes.c_int32, dp, dp,
+                                   ctypes.c_int32]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, dp, dp, dp, dp]
         lib.orc_merge.restype = None
@@ -66,7 +67,7 @@ def _ptr(a, ctype):
 
 def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pages_per_seq,
          num_pages, paged, elem_type, q_nope, q_rope, kv, block_table, seq_lens, sm_scale,
-         b_list, nthreads):
+         b_list, nthreads, h_list=None):
     lib = _load()
     shp = _Shape(VARIANT_IDS[variant], batch, num_q_heads, num_kv, d_nope, d_rope, page_size,
                  max_pages_per_seq, num_pages, 1 if paged else 0)
@@ -80,34 +81,39 @@ def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pag
         b_list = np.arange(batch, dtype=np.int32)
     b_list = np.ascontiguousarray(b_list, dtype=np.int32)
     nb = len(b_list)
-    out = np.zeros((nb, num_q_heads, d_nope), dtype=np.float64)
-    lse_rows = num_q_heads * num_kv if variant == "mlra" else num_q_heads
+    if h_list is not None:
+        h_list = np.ascontiguousarray(h_list, dtype=np.int32)
+    nh = num_q_heads if h_list is None else len(h_list)
+    out = np.zeros((nb, nh, d_nope), dtype=np.float64)
+    lse_rows = nh * num_kv if variant == "mlra" else nh
     lse = np.zeros((nb, lse_rows), dtype=np.float64)
     rc = lib.orc_decode(ctypes.byref(shp), elem_type, q_nope.ctypes.data,
                         None if q_rope_arr is None else q_rope_arr.ctypes.data, kv.ctypes.data,
                         None if bt is None else _ptr(bt, ctypes.c_int32), _ptr(seq_lens, ctypes.c_int32),
                         float(sm_scale), _ptr(b_list, ctypes.c_int32), nb,
+                        None if h_list is None else _ptr(h_list, ctypes.c_int32), nh,
                         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
                         int(nthreads or default_threads()))
     if rc != 0:
         raise RuntimeError(f"oracle failed with status {rc}")
     if variant == "mlra":
-        lse = lse.reshape(nb, num_q_heads, num_kv)
+        lse = lse.reshape(nb, nh, num_kv)
     return out, lse
 
 
-def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None):
+def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None):
     """fp64 decode attention of a workload dict (from ``workloads.make_inputs``).
 
-    Returns ``(out, lse)``: out ``[n_b][H][d_nope]`` float64 (MLRA: the sum
-    over branches), lse ``[n_b][H]`` (MLRA ``[n_b][H][R]``), natural log.
+    Returns ``(out, lse)``: out ``[n_b][n_h][d_nope]`` float64 (MLRA: the sum
+    over branches), lse ``[n_b][n_h]`` (MLRA ``[n_b][n_h][R]``), natural log.
+    ``b_list`` / ``h_list`` select sequences / heads (default: all).
     """
     s = inputs["shape"]
     scale = inputs["sm_scale"] if sm_scale is None else sm_scale
     return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
                 inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 0,
                 inputs["q_nope"], inputs["q_rope"], inputs["kv"], inputs["block_table"],
-                inputs["seq_lens"], scale, b_list, nthreads)
+                inputs["seq_lens"], scale, b_list, nthreads, h_list)
 
 
 def decode_f64(variant, num_kv, q_nope, q_rope, kv, seq_lens, sm_scale, block_table=None,

@@ -1,0 +1,274 @@
+// Host side of the C ABI declared in include/kvattn.h: argument validation,
+// launch planning, workspace layout and the two launches of one decode call.
+// Nothing here allocates device memory or reads it back, except
+// kvattn_get_device_error.
+#include <math.h>
+#include <string.h>
+
+#include "kvattn_internal.cuh"
+
+namespace kvattn {
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int validate(int32_t variant, const kvattn_params *p, Problem *pr)
+{
+    if (!p || !pr)
+        return KVATTN_ERR_INVALID_ARG;
+    if (variant < KVATTN_GQA || variant > KVATTN_MLRA)
+        return KVATTN_ERR_UNSUPPORTED;
+    if (p->batch < 1 || p->num_q_heads < 1 || p->num_kv < 1 || p->d_nope < 1 || p->d_rope < 0 ||
+        p->max_pages_per_seq < 1 || p->num_pages < 1 || p->max_seq_len < 0 || p->num_splits < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (p->out_dtype != KVATTN_OUT_BF16 && p->out_dtype != KVATTN_OUT_FP32)
+        return KVATTN_ERR_INVALID_ARG;
+    if (p->batch > 65535 || p->num_q_heads > 65535)
+        return KVATTN_ERR_UNSUPPORTED;
+    if (p->page_size != kPage)
+        return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)p->max_seq_len > (long long)p->max_pages_per_seq * kPage)
+        return KVATTN_ERR_INVALID_ARG;
+    if (p->d_nope % 8 || p->d_rope % 8)
+        return KVATTN_ERR_UNSUPPORTED;
+    if (p->d_nope > 512 || p->d_rope > 128)
+        return KVATTN_ERR_UNSUPPORTED;
+    const bool latent = variant == KVATTN_MLA || variant == KVATTN_GLA || variant == KVATTN_MLRA;
+    if (!latent && p->d_rope != 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if ((variant == KVATTN_MQA || variant == KVATTN_MLA) && p->num_kv != 1)
+        return KVATTN_ERR_INVALID_ARG;
+    if ((variant == KVATTN_GQA || variant == KVATTN_GLA) && p->num_q_heads % p->num_kv)
+        return KVATTN_ERR_INVALID_ARG;
+    if (variant == KVATTN_MLRA && p->num_kv > 16)
+        return KVATTN_ERR_UNSUPPORTED;
+    const long long row = latent ? (long long)p->num_kv * p->d_nope + p->d_rope
+                                 : (long long)p->num_kv * p->d_nope;
+    if (row > (1 << 20))
+        return KVATTN_ERR_UNSUPPORTED;
+
+    pr->variant = variant;
+    pr->B = p->batch;
+    pr->H = p->num_q_heads;
+    pr->NU = p->num_kv;
+    pr->dn = p->d_nope;
+    pr->dr = p->d_rope;
+    pr->Dk = p->d_nope + p->d_rope;
+    pr->Dv = p->d_nope;
+    pr->row = (int)row;
+    pr->latent = latent;
+    pr->mlra = variant == KVATTN_MLRA;
+    pr->HPU = pr->mlra ? pr->H : pr->H / pr->NU;
+    pr->HU = pr->mlra ? pr->H * pr->NU : pr->H;
+    pr->mpps = p->max_pages_per_seq;
+    pr->num_pages = p->num_pages;
+    pr->max_seq_len = p->max_seq_len;
+    pr->out_dtype = p->out_dtype;
+    pr->paged = true;
+    return KVATTN_OK;
+}
+
+// Heads per CTA of the generic kernel: the unit's heads, in chunks of at most 16.
+int generic_head_chunk(const Problem &pr)
+{
+    const int hpu = pr.HPU;
+    if (hpu >= 16)
+        return hpu % 16 == 0 ? 16 : 0;
+    if (hpu == 1 || hpu == 2 || hpu == 4 || hpu == 8)
+        return hpu;
+    return 0;
+}
+
+struct Plan {
+    kvattn_plan pub;
+    int head_chunk;
+    int head_chunks;
+    size_t lse_bytes;
+};
+
+int make_plan(const Problem &pr, int forced_splits, Plan *pl)
+{
+    memset(pl, 0, sizeof *pl);
+    const int hc = generic_head_chunk(pr);
+    if (!hc)
+        return KVATTN_ERR_UNSUPPORTED;
+    if (generic_smem_bytes(pr, hc) > 227 * 1024)
+        return KVATTN_ERR_UNSUPPORTED;
+    pl->head_chunk = hc;
+    pl->head_chunks = pr.HPU / hc;
+    const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
+    const long long base = (long long)pr.B * pr.NU * pl->head_chunks;
+    int splits;
+    if (forced_splits > 0) {
+        splits = forced_splits;
+    } else {
+        const long long target = 2LL * kNumSMs;
+        splits = (int)((target + base - 1) / base);
+    }
+    splits = splits < 1 ? 1 : splits;
+    splits = splits > max_pages ? max_pages : splits;
+    splits = splits > kMaxSplits ? kMaxSplits : splits;
+    const int pps = (max_pages + splits - 1) / splits;
+    splits = (max_pages + pps - 1) / pps;
+
+    pl->pub.kernel = KVATTN_KERNEL_GENERIC;
+    pl->pub.num_splits = splits;
+    pl->pub.pages_per_split = pps;
+    pl->pub.ctas = (int32_t)(base * splits);
+    pl->pub.launches = 2;
+    const size_t rows = (size_t)pr.B * splits * pr.HU;
+    pl->lse_bytes = align_up(rows * sizeof(float), 256);
+    pl->pub.workspace_bytes = kWsHeader + pl->lse_bytes + rows * pr.Dv * sizeof(float);
+    return KVATTN_OK;
+}
+
+}  // namespace
+}  // namespace kvattn
+
+using namespace kvattn;
+
+extern "C" int kvattn_version(void) { return 100; }
+
+extern "C" const char *kvattn_status_string(int status)
+{
+    switch (status) {
+    case KVATTN_OK: return "ok";
+    case KVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case KVATTN_ERR_UNSUPPORTED: return "unsupported problem";
+    case KVATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case KVATTN_ERR_MISALIGNED: return "misaligned pointer";
+    case KVATTN_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int kvattn_get_plan(int32_t variant, const kvattn_params *p, kvattn_plan *plan)
+{
+    if (!plan)
+        return KVATTN_ERR_INVALID_ARG;
+    Problem pr;
+    int st = validate(variant, p, &pr);
+    if (st)
+        return st;
+    Plan pl;
+    st = make_plan(pr, p->num_splits, &pl);
+    if (st)
+        return st;
+    *plan = pl.pub;
+    return KVATTN_OK;
+}
+
+extern "C" int kvattn_workspace_size(int32_t variant, const kvattn_params *p, size_t *bytes)
+{
+    if (!bytes)
+        return KVATTN_ERR_INVALID_ARG;
+    kvattn_plan plan;
+    const int st = kvattn_get_plan(variant, p, &plan);
+    if (st)
+        return st;
+    *bytes = (size_t)plan.workspace_bytes;
+    return KVATTN_OK;
+}
+
+extern "C" int kvattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace || workspace_bytes < kWsHeader)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256))
+        return KVATTN_ERR_MISALIGNED;
+    if (cudaMemsetAsync(workspace, 0, kWsHeader, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+    return KVATTN_OK;
+}
+
+extern "C" int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope,
+                             const void *q_rope, const void *kv_cache, const int32_t *block_table,
+                             const int32_t *seq_lens, float sm_scale, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    Problem pr;
+    int st = validate(variant, p, &pr);
+    if (st)
+        return st;
+    if (!q_nope || !kv_cache || !seq_lens || !out || !workspace)
+        return KVATTN_ERR_INVALID_ARG;
+    if (pr.dr > 0 && !q_rope)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!isfinite(sm_scale))
+        return KVATTN_ERR_INVALID_ARG;
+    if (!aligned(q_nope, 16) || (q_rope && !aligned(q_rope, 16)) || !aligned(kv_cache, 16) ||
+        !aligned(out, 16) || (lse && !aligned(lse, 4)) || !aligned(workspace, 256) ||
+        !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
+        return KVATTN_ERR_MISALIGNED;
+    Plan pl;
+    st = make_plan(pr, p->num_splits, &pl);
+    if (st)
+        return st;
+    if (workspace_bytes < pl.pub.workspace_bytes)
+        return KVATTN_ERR_WORKSPACE_TOO_SMALL;
+
+    char *ws = static_cast<char *>(workspace);
+    DecodeArgs a{};
+    a.q_nope = static_cast<const __nv_bfloat16 *>(q_nope);
+    a.q_rope = static_cast<const __nv_bfloat16 *>(q_rope);
+    a.kv = static_cast<const __nv_bfloat16 *>(kv_cache);
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.err = reinterpret_cast<int *>(ws);
+    a.plse = reinterpret_cast<float *>(ws + kWsHeader);
+    a.po = reinterpret_cast<float *>(ws + kWsHeader + pl.lse_bytes);
+    a.B = pr.B;
+    a.H = pr.H;
+    a.NU = pr.NU;
+    a.dn = pr.dn;
+    a.dr = pr.dr;
+    a.row = pr.row;
+    a.HPU = pr.HPU;
+    a.HU = pr.HU;
+    a.mpps = pr.mpps;
+    a.num_pages = pr.num_pages;
+    a.max_seq_len = pr.max_seq_len;
+    a.num_splits = pl.pub.num_splits;
+    a.pages_per_split = pl.pub.pages_per_split;
+    a.head_chunks = pl.head_chunks;
+    a.latent = pr.latent;
+    a.mlra = pr.mlra;
+    a.scale_log2 = sm_scale * 1.4426950408889634f;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_generic(a, pl.head_chunk, s) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+
+    CombineArgs c{};
+    c.po = a.po;
+    c.plse = a.plse;
+    c.out = out;
+    c.lse = lse;
+    c.B = pr.B;
+    c.H = pr.H;
+    c.NU = pr.NU;
+    c.Dv = pr.Dv;
+    c.HU = pr.HU;
+    c.num_splits = pl.pub.num_splits;
+    c.mlra = pr.mlra;
+    c.out_fp32 = pr.out_dtype == KVATTN_OUT_FP32;
+    if (launch_combine(c, s) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+    return KVATTN_OK;
+}
+
+extern "C" int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code)
+{
+    if (!workspace || !code)
+        return KVATTN_ERR_INVALID_ARG;
+    int32_t v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+    *code = v;
+    return KVATTN_OK;
+}

@@ -1,0 +1,163 @@
+"""Thin ctypes binding of libkvattn.so (include/kvattn.h).
+
+The functions carry the C names and only marshal arguments: device pointers
+are Python ints (``tensor.data_ptr()``), streams are ``cudaStream_t`` handles
+as ints (``torch.cuda.current_stream().cuda_stream``).  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.  If the
+library is missing, loading raises.
+
+``decode_tensors`` is a convenience that reads pointers and sizes from torch
+tensors and calls ``kvattn_decode``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvattn.so")
+
+KVATTN_GQA, KVATTN_MQA, KVATTN_MLA, KVATTN_GLA, KVATTN_MLRA = range(5)
+VARIANTS = {"gqa": KVATTN_GQA, "mqa": KVATTN_MQA, "mla": KVATTN_MLA, "gla": KVATTN_GLA,
+            "mlra": KVATTN_MLRA}
+KVATTN_OUT_BF16, KVATTN_OUT_FP32 = 0, 1
+KVATTN_OK = 0
+KVATTN_ERR_INVALID_ARG = -1
+KVATTN_ERR_UNSUPPORTED = -2
+KVATTN_ERR_WORKSPACE_TOO_SMALL = -3
+KVATTN_ERR_MISALIGNED = -4
+KVATTN_ERR_CUDA = -5
+KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1
+KVATTN_DEVERR_SEQ_TOO_LONG = 2
+KVATTN_DEVERR_WAIT_TIMEOUT = 4
+KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc"}
+
+EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
+           "kvattn_get_device_error", "kvattn_status_string", "kvattn_version")
+
+
+class kvattn_params(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "num_q_heads", "num_kv", "d_nope", "d_rope", "page_size", "max_pages_per_seq",
+        "num_pages", "max_seq_len", "num_splits", "out_dtype")]
+
+
+class kvattn_plan(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("num_splits", ctypes.c_int32),
+                ("pages_per_split", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_uint64)]
+
+
+class KvattnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {kvattn_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load():
+    """Load libkvattn.so (must have been built; see ``build.py``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with shared_kv_caches_b200.build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(kvattn_params)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.kvattn_get_plan.argtypes = [i32, P, ctypes.POINTER(kvattn_plan)]
+    lib.kvattn_workspace_size.argtypes = [i32, P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kvattn_workspace_init.argtypes = [vp, ctypes.c_size_t, vp]
+    lib.kvattn_decode.argtypes = [i32, P, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                  ctypes.c_size_t, vp]
+    lib.kvattn_get_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.kvattn_status_string.argtypes = [ctypes.c_int]
+    lib.kvattn_status_string.restype = ctypes.c_char_p
+    lib.kvattn_version.argtypes = []
+    for name in ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
+                 "kvattn_get_device_error", "kvattn_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def make_params(batch, num_q_heads, num_kv, d_nope, d_rope, max_pages_per_seq, num_pages,
+                max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64) -> kvattn_params:
+    return kvattn_params(int(batch), int(num_q_heads), int(num_kv), int(d_nope), int(d_rope),
+                         int(page_size), int(max_pages_per_seq), int(num_pages), int(max_seq_len),
+                         int(num_splits), int(out_dtype))
+
+
+def kvattn_version() -> int:
+    return load().kvattn_version()
+
+
+def kvattn_status_string(status: int) -> str:
+    return load().kvattn_status_string(int(status)).decode()
+
+
+def kvattn_get_plan(variant: int, params: kvattn_params) -> kvattn_plan:
+    plan = kvattn_plan()
+    st = load().kvattn_get_plan(int(variant), ctypes.byref(params), ctypes.byref(plan))
+    if st:
+        raise KvattnError(st, "kvattn_get_plan")
+    return plan
+
+
+def kvattn_workspace_size(variant: int, params: kvattn_params) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().kvattn_workspace_size(int(variant), ctypes.byref(params), ctypes.byref(n))
+    if st:
+        raise KvattnError(st, "kvattn_workspace_size")
+    return n.value
+
+
+def kvattn_workspace_init(workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return load().kvattn_workspace_init(workspace, workspace_bytes, stream)
+
+
+def kvattn_decode(variant, params, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale, out,
+                  lse, workspace, workspace_bytes, stream=0) -> int:
+    """Call the C entry point; returns its status (0 = enqueued)."""
+    return load().kvattn_decode(int(variant), ctypes.byref(params), q_nope, q_rope, kv_cache,
+                                block_table, seq_lens, float(sm_scale), out, lse, workspace,
+                                int(workspace_bytes), stream)
+
+
+def kvattn_get_device_error(workspace: int, stream: int = 0) -> int:
+    code = ctypes.c_int32(0)
+    st = load().kvattn_get_device_error(workspace, stream, ctypes.byref(code))
+    if st:
+        raise KvattnError(st, "kvattn_get_device_error")
+    return code.value
+
+
+# ----------------------------------------------------------------- torch glue
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def params_for(shape, max_pages_per_seq, num_pages, max_seq_len, num_splits=0) -> kvattn_params:
+    """Params of a ``workloads.Shape`` problem."""
+    return make_params(shape.batch, shape.num_q_heads, shape.num_kv, shape.d_nope, shape.d_rope,
+                       max_pages_per_seq, num_pages, max_seq_len, num_splits,
+                       KVATTN_OUT_FP32 if shape.out_dtype == "fp32" else KVATTN_OUT_BF16,
+                       shape.page_size)
+
+
+def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, sm_scale, out, lse,
+                   workspace, stream=None) -> None:
+    """``kvattn_decode`` on torch tensors; raises on a non-zero status."""
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+    st = kvattn_decode(variant, params, _ptr(q_nope), _ptr(q_rope), _ptr(kv), _ptr(block_table),
+                       _ptr(seq_lens), sm_scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                       workspace.numel() * workspace.element_size(), stream)
+    if st:
+        raise KvattnError(st, "kvattn_decode")

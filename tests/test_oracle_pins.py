@@ -411,3 +411,11 @@ def test_sample_of_sequences_matches_full(oracle_mod):
     o2, l2 = oracle_mod.decode(x, b_list=[3, 1])
     np.testing.assert_array_equal(o2, out[[3, 1]])
     np.testing.assert_array_equal(l2, lse[[3, 1]])
+    o3, l3 = oracle_mod.decode(x, b_list=[2], h_list=[5, 0])
+    np.testing.assert_array_equal(o3[0], out[2, [5, 0]])
+    np.testing.assert_array_equal(l3[0], lse[2, [5, 0]])
+    y = W.make_inputs(W.Shape("mlra", 2, 4, 3, 16, 8, (10, 90)), seed=3)
+    out, lse = oracle_mod.decode(y)
+    o4, l4 = oracle_mod.decode(y, b_list=[1], h_list=[3])
+    np.testing.assert_array_equal(o4[0, 0], out[1, 3])
+    np.testing.assert_array_equal(l4[0, 0], lse[1, 3])
