@@ -163,6 +163,17 @@ int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope, c
                   float sm_scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
                   void *stream);
 
+/* kvattn_decode that also records caller-created cudaEvent_t handles on
+ * `stream`: events[0] before the split pass, events[1] between the split pass
+ * and the combine pass, events[2] after the combine pass (a NULL entry is
+ * skipped; events may be NULL).  Used to time each pass on the launching
+ * stream.  Same arguments, statuses and results as kvattn_decode. */
+int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_nope,
+                        const void *q_rope, const void *kv_cache, const int32_t *block_table,
+                        const int32_t *seq_lens, float sm_scale, void *out, float *lse,
+                        void *workspace, size_t workspace_bytes, void *stream,
+                        void *const *events);
+
 /* Copy the device error word to *code (0 = none, else kvattn_device_error
  * bits).  Synchronises `stream`.  Returns KVATTN_ERR_CUDA if the copy
  * failed. */

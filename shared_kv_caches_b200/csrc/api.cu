@@ -183,10 +183,11 @@ extern "C" int kvattn_workspace_init(void *workspace, size_t workspace_bytes, vo
     return KVATTN_OK;
 }
 
-extern "C" int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope,
-                             const void *q_rope, const void *kv_cache, const int32_t *block_table,
-                             const int32_t *seq_lens, float sm_scale, void *out, float *lse,
-                             void *workspace, size_t workspace_bytes, void *stream)
+extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_nope,
+                                   const void *q_rope, const void *kv_cache,
+                                   const int32_t *block_table, const int32_t *seq_lens,
+                                   float sm_scale, void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, void *stream, void *const *events)
 {
     Problem pr;
     int st = validate(variant, p, &pr);
@@ -238,7 +239,15 @@ extern "C" int kvattn_decode(int32_t variant, const kvattn_params *p, const void
     a.scale_log2 = sm_scale * 1.4426950408889634f;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto mark = [&](int i) {
+        return !(events && events[i]) ||
+               cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s) == cudaSuccess;
+    };
+    if (!mark(0))
+        return KVATTN_ERR_CUDA;
     if (launch_generic(a, pl.head_chunk, s) != cudaSuccess)
+        return KVATTN_ERR_CUDA;
+    if (!mark(1))
         return KVATTN_ERR_CUDA;
 
     CombineArgs c{};
@@ -256,7 +265,18 @@ extern "C" int kvattn_decode(int32_t variant, const kvattn_params *p, const void
     c.out_fp32 = pr.out_dtype == KVATTN_OUT_FP32;
     if (launch_combine(c, s) != cudaSuccess)
         return KVATTN_ERR_CUDA;
+    if (!mark(2))
+        return KVATTN_ERR_CUDA;
     return KVATTN_OK;
+}
+
+extern "C" int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope,
+                             const void *q_rope, const void *kv_cache, const int32_t *block_table,
+                             const int32_t *seq_lens, float sm_scale, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    return kvattn_decode_timed(variant, p, q_nope, q_rope, kv_cache, block_table, seq_lens,
+                               sm_scale, out, lse, workspace, workspace_bytes, stream, nullptr);
 }
 
 extern "C" int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code)

@@ -48,7 +48,7 @@ class DeviceProblem:
         self.lse = torch.empty(s.lse_shape(), dtype=torch.float32, device=self.device)
 
     def run(self, stream=None, out=None, lse=None, q_nope=None, q_rope=None, seq_lens=None,
-            block_table=None):
+            block_table=None, events=None):
         """Enqueue one decode call (optionally on other q / out buffers)."""
         K.decode_tensors(self.variant, self.params,
                          self.q_nope if q_nope is None else q_nope,
@@ -59,7 +59,10 @@ class DeviceProblem:
                          self.sm_scale,
                          self.out if out is None else out,
                          self.lse if lse is None else lse,
-                         self.workspace, stream)
+                         self.workspace, stream, events)
+
+    def plan_kernel_name(self) -> str:
+        return K.KERNEL_NAMES.get(int(self.plan.kernel), str(self.plan.kernel))
 
     def device_error(self) -> int:
         import torch

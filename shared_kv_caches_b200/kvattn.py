@@ -34,7 +34,7 @@ KVATTN_DEVERR_WAIT_TIMEOUT = 4
 KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc"}
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
-           "kvattn_get_device_error", "kvattn_status_string", "kvattn_version")
+           "kvattn_decode_timed", "kvattn_get_device_error", "kvattn_status_string", "kvattn_version")
 
 
 class kvattn_params(ctypes.Structure):
@@ -74,12 +74,14 @@ def load():
     lib.kvattn_workspace_init.argtypes = [vp, ctypes.c_size_t, vp]
     lib.kvattn_decode.argtypes = [i32, P, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                                   ctypes.c_size_t, vp]
+    lib.kvattn_decode_timed.argtypes = [i32, P, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                        ctypes.c_size_t, vp, ctypes.POINTER(ctypes.c_void_p)]
     lib.kvattn_get_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
     lib.kvattn_status_string.argtypes = [ctypes.c_int]
     lib.kvattn_status_string.restype = ctypes.c_char_p
     lib.kvattn_version.argtypes = []
     for name in ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
-                 "kvattn_get_device_error", "kvattn_version"):
+                 "kvattn_decode_timed", "kvattn_get_device_error", "kvattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -128,6 +130,15 @@ def kvattn_decode(variant, params, q_nope, q_rope, kv_cache, block_table, seq_le
                                 int(workspace_bytes), stream)
 
 
+def kvattn_decode_timed(variant, params, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale,
+                        out, lse, workspace, workspace_bytes, stream, events) -> int:
+    """``kvattn_decode`` recording three cudaEvent_t handles (ints or None)."""
+    ev = (ctypes.c_void_p * 3)(*[e for e in events])
+    return load().kvattn_decode_timed(int(variant), ctypes.byref(params), q_nope, q_rope, kv_cache,
+                                      block_table, seq_lens, float(sm_scale), out, lse, workspace,
+                                      int(workspace_bytes), stream, ev)
+
+
 def kvattn_get_device_error(workspace: int, stream: int = 0) -> int:
     code = ctypes.c_int32(0)
     st = load().kvattn_get_device_error(workspace, stream, ctypes.byref(code))
@@ -151,13 +162,21 @@ def params_for(shape, max_pages_per_seq, num_pages, max_seq_len, num_splits=0) -
 
 
 def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, sm_scale, out, lse,
-                   workspace, stream=None) -> None:
-    """``kvattn_decode`` on torch tensors; raises on a non-zero status."""
+                   workspace, stream=None, events=None) -> None:
+    """``kvattn_decode`` on torch tensors; raises on a non-zero status.
+
+    ``events``: three ``torch.cuda.Event`` (or None) recorded around the split
+    pass and the combine pass on the launching stream.
+    """
     if stream is None:
         import torch
         stream = torch.cuda.current_stream(q_nope.device).cuda_stream
-    st = kvattn_decode(variant, params, _ptr(q_nope), _ptr(q_rope), _ptr(kv), _ptr(block_table),
-                       _ptr(seq_lens), sm_scale, _ptr(out), _ptr(lse), _ptr(workspace),
-                       workspace.numel() * workspace.element_size(), stream)
+    args = (variant, params, _ptr(q_nope), _ptr(q_rope), _ptr(kv), _ptr(block_table), _ptr(seq_lens),
+            sm_scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            stream)
+    if events is None:
+        st = kvattn_decode(*args)
+    else:
+        st = kvattn_decode_timed(*args, [None if e is None else e.cuda_event for e in events])
     if st:
         raise KvattnError(st, "kvattn_decode")
