@@ -175,6 +175,13 @@ def run_ours(args, rank, world, local):
     K = args.steps
     step_ev = [(Ev(enable_timing=True), Ev(enable_timing=True)) for _ in range(K)]
     kern_ev = [[[Ev(enable_timing=True) for _ in range(3)] for _ in probs] for _ in range(K)]
+    # torch creates a CUDA event on its first record(); do that here so the
+    # handles the library records inside the timed region exist
+    for per_step in kern_ev:
+        for trio in per_step:
+            for e in trio:
+                e.record()
+    torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(dev)
     bus = None
     if all(hasattr(props, a) for a in ("pci_domain_id", "pci_bus_id", "pci_device_id")):
