@@ -174,6 +174,43 @@ int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_n
                         void *workspace, size_t workspace_bytes, void *stream,
                         void *const *events);
 
+/*
+ * Size of the device scratch array behind kvattn_decode_noalloc (32 MiB).
+ */
+#define KVATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * kvattn_decode_noalloc -- the same decode attention for callers that cannot
+ * allocate device memory.  The pages describe no such interface; it has no
+ * counterpart there.
+ *
+ * Who needs it: callers that cannot hand the library a workspace, because
+ * they may not call cudaMalloc at all -- a serving engine that has already
+ * reserved all of HBM for its own cache pool, a plugin host that gives a
+ * library only its input and output buffers, or a latency-critical path where
+ * an allocation (which can synchronise the device) is not acceptable.
+ *
+ * The caller passes the inputs and outputs exactly as for kvattn_decode
+ * (same layouts, alignment and statuses) but no workspace.  The scratch lives
+ * in one device array of KVATTN_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ * Nothing is allocated by this call.  A problem whose workspace does not fit
+ * is run with fewer parts per context when num_splits is 0; if it still does
+ * not fit, or a forced num_splits does not fit, the call returns
+ * KVATTN_ERR_WORKSPACE_TOO_SMALL and enqueues nothing.
+ *
+ * The first call on a device (that device current) looks up the array's
+ * device address; make that first call before any stream capture.  All calls
+ * share the one array, which keeps the last call's contents: calls ordered on
+ * one stream are safe, calls that overlap on the GPU race on it.  Each call
+ * clears the device error word at its start; device_error (device memory, 4
+ * bytes, may be NULL) receives that call's kvattn_device_error bits.
+ */
+int kvattn_decode_noalloc(int32_t variant, const kvattn_params *p, const void *q_nope,
+                          const void *q_rope, const void *kv_cache, const int32_t *block_table,
+                          const int32_t *seq_lens, float sm_scale, void *out, float *lse,
+                          int32_t *device_error, void *stream);
+
 /* Copy the device error word to *code (0 = none, else kvattn_device_error
  * bits).  Synchronises `stream`.  Returns KVATTN_ERR_CUDA if the copy
  * failed. */

@@ -34,7 +34,9 @@ KVATTN_DEVERR_WAIT_TIMEOUT = 4
 KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc"}
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
-           "kvattn_decode_timed", "kvattn_get_device_error", "kvattn_status_string", "kvattn_version")
+           "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
+           "kvattn_status_string", "kvattn_version")
+KVATTN_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class kvattn_params(ctypes.Structure):
@@ -76,12 +78,14 @@ def load():
                                   ctypes.c_size_t, vp]
     lib.kvattn_decode_timed.argtypes = [i32, P, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                                         ctypes.c_size_t, vp, ctypes.POINTER(ctypes.c_void_p)]
+    lib.kvattn_decode_noalloc.argtypes = [i32, P, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp]
     lib.kvattn_get_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
     lib.kvattn_status_string.argtypes = [ctypes.c_int]
     lib.kvattn_status_string.restype = ctypes.c_char_p
     lib.kvattn_version.argtypes = []
     for name in ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
-                 "kvattn_decode_timed", "kvattn_get_device_error", "kvattn_version"):
+                 "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
+                 "kvattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -137,6 +141,15 @@ def kvattn_decode_timed(variant, params, q_nope, q_rope, kv_cache, block_table, 
     return load().kvattn_decode_timed(int(variant), ctypes.byref(params), q_nope, q_rope, kv_cache,
                                       block_table, seq_lens, float(sm_scale), out, lse, workspace,
                                       int(workspace_bytes), stream, ev)
+
+
+def kvattn_decode_noalloc(variant, params, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale,
+                          out, lse, device_error, stream=0) -> int:
+    """Decode without a caller workspace (for callers that cannot allocate
+    device memory); scratch is the library's own fixed device array."""
+    return load().kvattn_decode_noalloc(int(variant), ctypes.byref(params), q_nope, q_rope, kv_cache,
+                                        block_table, seq_lens, float(sm_scale), out, lse, device_error,
+                                        stream)
 
 
 def kvattn_get_device_error(workspace: int, stream: int = 0) -> int:
