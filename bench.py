@@ -58,6 +58,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--splits", type=int, default=0, help="force parts per context (0: library choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     a = ap.parse_args(argv)
@@ -149,7 +150,7 @@ def run_ours(args, rank, world, local):
     names = problem_names(args.workload)
     seed = BU.rank_seed(args.seed, rank)
     inputs = [W.make_inputs(W.WORKLOADS[n], seed=seed) for n in names]
-    probs = [DeviceProblem(x, dev) for x in inputs]
+    probs = [DeviceProblem(x, dev, num_splits=args.splits) for x in inputs]
     costs = [BU.step_cost(x["shape"], x["seq_lens"]) for x in inputs]
     batch = inputs[0]["shape"].batch
     flush = torch.empty(252 * 1024 * 1024, dtype=torch.uint8, device=dev)

@@ -88,32 +88,50 @@ struct Plan {
     size_t lse_bytes;
 };
 
-int make_plan(const Problem &pr, int forced_splits, Plan *pl)
+// Parts per context: forced, or enough CTAs for several waves over the SMs
+// (counted from the longest context, the only length the host knows).
+int choose_splits(int forced, long long units, int max_pages, long long target_ctas, int min_pages_per_split)
 {
-    memset(pl, 0, sizeof *pl);
-    const int hc = generic_head_chunk(pr);
-    if (!hc)
-        return KVATTN_ERR_UNSUPPORTED;
-    if (generic_smem_bytes(pr, hc) > 227 * 1024)
-        return KVATTN_ERR_UNSUPPORTED;
-    pl->head_chunk = hc;
-    pl->head_chunks = pr.HPU / hc;
-    const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
-    const long long base = (long long)pr.B * pr.NU * pl->head_chunks;
     int splits;
-    if (forced_splits > 0) {
-        splits = forced_splits;
+    if (forced > 0) {
+        splits = forced;
     } else {
-        const long long target = 2LL * kNumSMs;
-        splits = (int)((target + base - 1) / base);
+        splits = (int)((target_ctas + units - 1) / units);
+        const int cap = (max_pages + min_pages_per_split - 1) / min_pages_per_split;
+        splits = splits > cap ? cap : splits;
     }
     splits = splits < 1 ? 1 : splits;
     splits = splits > max_pages ? max_pages : splits;
     splits = splits > kMaxSplits ? kMaxSplits : splits;
+    return splits;
+}
+
+int make_plan(const Problem &pr, int forced_splits, Plan *pl)
+{
+    memset(pl, 0, sizeof *pl);
+    const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
+    long long base;
+    int splits;
+    if (gqa_supported(pr)) {
+        pl->pub.kernel = KVATTN_KERNEL_GQA;
+        pl->head_chunk = 4;
+        pl->head_chunks = 1;
+        base = (long long)pr.B * pr.NU;
+        splits = choose_splits(forced_splits, base, max_pages, 4LL * 3 * kNumSMs, 4);
+    } else {
+        const int hc = generic_head_chunk(pr);
+        if (!hc)
+            return KVATTN_ERR_UNSUPPORTED;
+        if (generic_smem_bytes(pr, hc) > 227 * 1024)
+            return KVATTN_ERR_UNSUPPORTED;
+        pl->pub.kernel = KVATTN_KERNEL_GENERIC;
+        pl->head_chunk = hc;
+        pl->head_chunks = pr.HPU / hc;
+        base = (long long)pr.B * pr.NU * pl->head_chunks;
+        splits = choose_splits(forced_splits, base, max_pages, 2LL * kNumSMs, 1);
+    }
     const int pps = (max_pages + splits - 1) / splits;
     splits = (max_pages + pps - 1) / pps;
-
-    pl->pub.kernel = KVATTN_KERNEL_GENERIC;
     pl->pub.num_splits = splits;
     pl->pub.pages_per_split = pps;
     pl->pub.ctas = (int32_t)(base * splits);
@@ -245,7 +263,9 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     };
     if (!mark(0))
         return KVATTN_ERR_CUDA;
-    if (launch_generic(a, pl.head_chunk, s) != cudaSuccess)
+    const cudaError_t le = pl.pub.kernel == KVATTN_KERNEL_GQA ? launch_gqa(a, s)
+                                                            : launch_generic(a, pl.head_chunk, s);
+    if (le != cudaSuccess)
         return KVATTN_ERR_CUDA;
     if (!mark(1))
         return KVATTN_ERR_CUDA;

@@ -59,5 +59,7 @@ __device__ __forceinline__ void raise_error(int *err, int bit) { atomicOr(err, b
 cudaError_t launch_generic(const DecodeArgs &a, int head_chunk, cudaStream_t st);
 size_t generic_smem_bytes(const Problem &pr, int head_chunk);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
+bool gqa_supported(const Problem &pr);
+cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st);
 
 }  // namespace kvattn
