@@ -118,6 +118,12 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunks = 1;
         base = (long long)pr.B * pr.NU;
         splits = choose_splits(forced_splits, base, max_pages, 4LL * 3 * kNumSMs, 4);
+    } else if (mqa_mma_supported(pr)) {
+        pl->pub.kernel = KVATTN_KERNEL_MQA_TC;
+        pl->head_chunk = 32;
+        pl->head_chunks = 1;
+        base = (long long)pr.B * pr.NU;
+        splits = choose_splits(forced_splits, base, max_pages, 4LL * kNumSMs, 2);
     } else {
         const int hc = generic_head_chunk(pr);
         if (!hc)
@@ -263,8 +269,12 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     };
     if (!mark(0))
         return KVATTN_ERR_CUDA;
-    const cudaError_t le = pl.pub.kernel == KVATTN_KERNEL_GQA ? launch_gqa(a, s)
-                                                            : launch_generic(a, pl.head_chunk, s);
+    cudaError_t le;
+    switch (pl.pub.kernel) {
+    case KVATTN_KERNEL_GQA: le = launch_gqa(a, s); break;
+    case KVATTN_KERNEL_MQA_TC: le = launch_mqa_mma(a, s); break;
+    default: le = launch_generic(a, pl.head_chunk, s); break;
+    }
     if (le != cudaSuccess)
         return KVATTN_ERR_CUDA;
     if (!mark(1))

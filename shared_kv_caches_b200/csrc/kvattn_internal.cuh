@@ -61,5 +61,7 @@ size_t generic_smem_bytes(const Problem &pr, int head_chunk);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 bool gqa_supported(const Problem &pr);
 cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st);
+bool mqa_mma_supported(const Problem &pr);
+cudaError_t launch_mqa_mma(const DecodeArgs &a, cudaStream_t st);
 
 }  // namespace kvattn
