@@ -112,7 +112,14 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
     const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
     long long base;
     int splits;
-    if (gqa_supported(pr)) {
+    const int tc_slots = latent_tc_slots(pr);
+    if (tc_slots > 0) {
+        pl->pub.kernel = KVATTN_KERNEL_LATENT_TC;
+        pl->head_chunk = 128;
+        pl->head_chunks = tc_slots;
+        base = (long long)pr.B * tc_slots;
+        splits = choose_splits(forced_splits, base, max_pages, 4LL * kNumSMs, pr.mlra ? 16 : 64);
+    } else if (gqa_supported(pr)) {
         pl->pub.kernel = KVATTN_KERNEL_GQA;
         pl->head_chunk = 4;
         pl->head_chunks = 1;
@@ -273,6 +280,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     switch (pl.pub.kernel) {
     case KVATTN_KERNEL_GQA: le = launch_gqa(a, s); break;
     case KVATTN_KERNEL_MQA_TC: le = launch_mqa_mma(a, s); break;
+    case KVATTN_KERNEL_LATENT_TC: le = launch_latent_tc(a, pr, s); break;
     default: le = launch_generic(a, pl.head_chunk, s); break;
     }
     if (le != cudaSuccess)

@@ -1,0 +1,447 @@
+// Latent decode on the 5th-generation tensor cores: absorbed MLA, GLA and
+// MLRA.
+//
+// Every query head scores the same cached latent rows (MLRA page: after
+// absorption MLA decodes as one 576-wide MQA head; GLA page: one latent head
+// per query group; MLRA page: the latent split into branches attended on
+// their own), so the scores and P.V are real [128 heads x K] x [K x tokens]
+// contractions and run as tcgen05 MMAs with fp32 accumulators in TMEM.
+//
+// One CTA owns (part s of the context, slot, sequence b).  A slot is a value
+// half for MLA (the 128 x 512 fp32 output would fill all 512 TMEM columns, so
+// two CTAs each keep 256 value columns and both form the full scores), a
+// latent group for GLA (its 64 heads padded to the MMA's 128 rows) and a
+// branch for MLRA.  Key columns of the slot are [latent slice | shared rope
+// key], each a 64-column box of the page row.
+//
+// Warp roles (192 threads):
+//   warp 0     TMEM allocation; one thread streams each tile's key boxes into
+//              a STAGES-deep shared-memory ring with 2-D TMA loads (128-byte
+//              swizzle, completion on kv_full)
+//   warp 1     one thread issues S_j = Q K_j^T into one of two TMEM score
+//              buffers, then P_{j-1} V_{j-1} into the TMEM output; the warp
+//              zeroes the rows of a tile past the context first (0 * NaN
+//              would poison the MMA)
+//   warps 2-5  one thread per head row: read S_j from TMEM, online softmax in
+//              fp32 (base 2) with a lazy rescale (the reference max moves
+//              only when a score exceeds it by more than 2^8, so O is
+//              rarely touched), write P_j as bf16 into the score buffer it
+//              came from (the A operand of the P.V MMA), and at the end
+//              normalise O and write the part result and its lse.
+// Every wait is bounded; a wait that gives up sets an error bit and the CTA
+// drains its own copies and MMAs before it frees TMEM and exits.
+#include <math.h>
+
+#include "kvattn_internal.cuh"
+#include "sm100.cuh"
+
+namespace kvattn {
+
+namespace {
+
+constexpr int kRows = 128;                 // MMA M: query-head rows
+constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kQChunkBytes = kRows * 128;  // 128 rows x 64 bf16, 128-byte swizzle
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kRescaleThreshold = 8.f;   // log2 units
+
+template <int T, int NKB, int STAGES>
+struct LatentSmem {
+    static constexpr int kBoxBytes = T * 128;
+    static constexpr int kStageBytes = NKB * kBoxBytes;
+    unsigned char q[NKB][kQChunkBytes];
+    unsigned char kv[STAGES][kStageBytes];
+    uint64_t kv_full[STAGES];
+    uint64_t kv_empty[STAGES];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_ready;
+    uint64_t q_ready;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+};
+
+struct TileInfo {
+    long long page;
+    int off;    // token offset of the tile inside its page
+    int ntok;   // context tokens in the tile (0 if the page id is bad)
+};
+
+template <int T>
+__device__ __forceinline__ TileInfo tile_info(const DecodeArgs &a, int b, int L, int p0, int j)
+{
+    TileInfo ti;
+    const int tok0 = p0 * kPage + j * T;
+    const int pi = tok0 / kPage;
+    ti.off = tok0 % kPage;
+    ti.page = a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
+    const bool ok = ti.page >= 0 && ti.page < a.num_pages;
+    ti.ntok = ok ? min(T, L - tok0) : 0;
+    return ti;
+}
+
+template <int T, int NKB, int NVB, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    latent_tc_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a)
+{
+    using Smem = LatentSmem<T, NKB, STAGES>;
+    constexpr int kBoxBytes = Smem::kBoxBytes;
+    constexpr int kDvSlot = NVB * 64;                            // value columns of this CTA
+    constexpr uint32_t kTmemCols = (2 * T + kDvSlot) <= 256 ? 256 : 512;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kRows, T, false, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kRows, kDvSlot, false, true);
+
+    extern __shared__ unsigned char smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+    const bool mla = !a.mlra && a.NU == 1;
+    const int dn_boxes = a.dn / 64;
+
+    int L = a.seq_lens[b];
+    if (L > a.max_seq_len) {
+        if (threadIdx.x == 0 && split == 0 && slot == 0)
+            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
+        L = a.max_seq_len;
+    }
+    L = max(L, 0);
+    const int p0 = split * a.pages_per_split;
+    const int tok_end = min(L, (p0 + a.pages_per_split) * kPage);
+    const int n = tok_end > p0 * kPage ? (tok_end - p0 * kPage + T - 1) / T : 0;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(&S.kv_full[st], 1);
+            mbar_init(&S.kv_empty[st], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.s_full[i], 1);
+            mbar_init(&S.p_full[i], kSoftmaxThreads);
+        }
+        mbar_init(&S.o_ready, 1);
+        mbar_init(&S.q_ready, kSoftmaxThreads);
+        mbar_init(&S.mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0)
+        tmem_alloc(&S.tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = S.tmem_base;
+    const uint32_t tS = tbase;                 // 2 score / probability buffers of T columns
+    const uint32_t tO = tbase + 2 * T;         // kDvSlot output columns
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA
+        if (lane == 0 && n > 0) {
+            prefetch_tmap(&kv_map);
+            const int unit_col0 = mla ? 0 : slot * a.dn;
+            int issued = 0;
+            for (int j = 0; j < n; ++j) {
+                const int st = j % STAGES;
+                if (j >= STAGES && !mbar_wait(&S.kv_empty[st], ((j / STAGES) - 1) & 1)) {
+                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                    break;
+                }
+                const TileInfo ti = tile_info<T>(a, b, L, p0, j);
+                issued = j + 1;
+                if (ti.ntok == 0) {
+                    if (slot == 0 && ti.off == 0)
+                        raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);
+                    mbar_arrive(&S.kv_full[st]);
+                    continue;
+                }
+                mbar_arrive_expect_tx(&S.kv_full[st], Smem::kStageBytes);
+                const int y = (int)(ti.page * kPage) + ti.off;
+#pragma unroll
+                for (int i = 0; i < NKB; ++i) {
+                    const int col = i < dn_boxes ? unit_col0 + 64 * i : a.NU * a.dn + 64 * (i - dn_boxes);
+                    tma_load_2d(S.kv[st] + i * kBoxBytes, &kv_map, col, y, &S.kv_full[st]);
+                }
+            }
+            // every copy this thread started has landed before the CTA can exit
+            for (int st = 0; st < STAGES && st < issued; ++st) {
+                const int jl = st + ((issued - 1 - st) / STAGES) * STAGES;
+                if (!mbar_wait(&S.kv_full[st], (jl / STAGES) & 1))
+                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA
+        const uint32_t qbase = smem_u32(&S.q[0][0]);
+        bool ok = mbar_wait(&S.q_ready, 0);
+        tc_fence_after();
+        auto issue_pv = [&](int t) -> bool {
+            if (!mbar_wait(&S.p_full[t & 1], (t >> 1) & 1))
+                return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t vbase = smem_u32(S.kv[t % STAGES]) + (mla ? slot * NVB : 0) * kBoxBytes;
+#pragma unroll
+                for (int k = 0; k < T / 16; ++k) {
+                    const uint64_t vd = smem_desc(vbase + k * 16 * 128, kBoxBytes, 1024, 2);
+                    umma_ts(tO, tS + (t & 1) * T + 8 * k, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
+                }
+                umma_commit(&S.o_ready);
+                umma_commit(&S.kv_empty[t % STAGES]);
+            }
+            __syncwarp();
+            return true;
+        };
+        int j = 0;
+        for (; ok && j < n; ++j) {
+            const int st = j % STAGES;
+            if (!mbar_wait(&S.kv_full[st], (j / STAGES) & 1)) {
+                ok = false;
+                break;
+            }
+            const TileInfo ti = tile_info<T>(a, b, L, p0, j);
+            if (ti.ntok < T) {
+                // zero the rows past the context in every key box of the stage
+                const int rows = T - ti.ntok;
+                for (int idx = lane; idx < rows * NKB * 8; idx += 32) {
+                    const int box = idx / (rows * 8), rem = idx % (rows * 8);
+                    const int row = ti.ntok + rem / 8, piece = rem % 8;
+                    *reinterpret_cast<uint4 *>(S.kv[st] + box * kBoxBytes + row * 128 + piece * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t kbase = smem_u32(S.kv[st]);
+#pragma unroll
+                for (int kb = 0; kb < NKB; ++kb) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t qd = smem_desc(qbase + kb * kQChunkBytes + k * 32, 16, 1024, 2);
+                        const uint64_t kd = smem_desc(kbase + kb * kBoxBytes + k * 32, 16, 1024, 2);
+                        umma_ss(tS + (j & 1) * T, qd, kd, kIdescS, (kb | k) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&S.s_full[j & 1]);
+            }
+            __syncwarp();
+            if (j >= 1 && !issue_pv(j - 1)) {
+                ok = false;
+                break;
+            }
+        }
+        if (ok && n > 0 && !issue_pv(n - 1))
+            ok = false;
+        if (!ok && lane == 0)
+            raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+        // every MMA this thread issued has completed before TMEM is freed
+        if (lane == 0)
+            umma_commit(&S.mma_done);
+        __syncwarp();
+        if (!mbar_wait(&S.mma_done, 0) && lane == 0)
+            raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int quarter = warp & 3;
+        const int h = quarter * 32 + lane;                      // head row = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const int rows_used = a.mlra || mla ? a.H : a.HPU;     // GLA: the group's heads
+        {
+            // Q row h of this slot: [latent query slice | rope query], swizzled
+            const __nv_bfloat16 *qn = nullptr, *qr = nullptr;
+            if (h < rows_used) {
+                size_t row;
+                if (a.mlra)
+                    row = ((size_t)b * a.H + h) * a.NU + slot;
+                else if (mla)
+                    row = (size_t)b * a.H + h;
+                else
+                    row = (size_t)b * a.H + (size_t)slot * a.HPU + h;
+                qn = a.q_nope + row * a.dn;
+                qr = a.q_rope + row * a.dr;
+            }
+#pragma unroll 1
+            for (int kb = 0; kb < NKB; ++kb) {
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (qn)
+                        v = kb < dn_boxes ? *reinterpret_cast<const uint4 *>(qn + 64 * kb + 8 * p)
+                                          : *reinterpret_cast<const uint4 *>(qr + 64 * (kb - dn_boxes) + 8 * p);
+                    *reinterpret_cast<uint4 *>(&S.q[kb][h * 128 + ((p ^ (h & 7)) << 4)]) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&S.q_ready);
+        }
+
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int sb = j & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&S.s_full[sb], (j >> 1) & 1));
+            if (!ok)
+                break;
+            tc_fence_after();
+            float s[T];
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int c = 0; c < T / 32; ++c) {
+                    tmem_ld32(tS + lane_addr + sb * T + 32 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        s[32 * c + i] = __uint_as_float(r[i]);
+                }
+            }
+            const TileInfo ti = tile_info<T>(a, b, L, p0, j);
+            float mt = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < T; ++i) {
+                s[i] = i < ti.ntok ? s[i] * a.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, s[i]);
+            }
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mt > m_ref + kRescaleThreshold) {
+                if (m_ref != -INFINITY) {
+                    alpha = exp2f(m_ref - mt);
+                    rescale = true;
+                }
+                m_ref = mt;
+            }
+            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+            float ps = 0.f;
+            uint32_t pk[T / 2];
+#pragma unroll
+            for (int i = 0; i < T / 2; ++i) {
+                const float e0 = exp2f(s[2 * i] - m_use), e1 = exp2f(s[2 * i + 1] - m_use);
+                ps += e0 + e1;
+                const __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
+                pk[i] = *reinterpret_cast<const uint32_t *>(&v2);
+            }
+            l = l * alpha + ps;
+#pragma unroll
+            for (int c = 0; c < T / 32; ++c)
+                tmem_st16(tS + lane_addr + sb * T + 16 * c, pk + 16 * c);
+            // TMEM accesses are warp-wide: rescale the whole warp's rows when any needs it
+            if (__any_sync(0xffffffffu, rescale)) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (j - 1) & 1));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                uint32_t r[32];
+#pragma unroll 1
+                for (int c = 0; c < kDvSlot / 32; ++c) {
+                    tmem_ld32(tO + lane_addr + 32 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(tO + lane_addr + 32 * c, r);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&S.p_full[sb]);
+        }
+        if (!ok && lane == 0)
+            raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+
+        // part result: O / l and lse for this row
+        bool have = false;
+        if (ok && n > 0) {
+            have = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (n - 1) & 1));
+            if (!have && lane == 0)
+                raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+            tc_fence_after();
+        }
+        const bool valid = h < rows_used;
+        int hu, col0;
+        if (a.mlra) {
+            hu = h * a.NU + slot;
+            col0 = 0;
+        } else if (mla) {
+            hu = h;
+            col0 = slot * kDvSlot;
+        } else {
+            hu = slot * a.HPU + h;
+            col0 = 0;
+        }
+        const size_t prow = ((size_t)b * a.num_splits + split) * a.HU + (valid ? hu : 0);
+        float *dst = a.po + prow * a.dn + col0;
+        const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+        uint32_t r[32];
+#pragma unroll 1
+        for (int c = 0; c < kDvSlot / 32; ++c) {
+            if (have)
+                tmem_ld32(tO + lane_addr + 32 * c, r);
+            if (valid) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (have)
+                        v = make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                                        __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
+                    *reinterpret_cast<float4 *>(dst + 32 * c + i) = v;
+                }
+            }
+        }
+        if (valid && (!mla || slot == 0))
+            a.plse[prow] = (have && l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+    }
+    __syncwarp();
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        tmem_dealloc(tbase, kTmemCols);
+}
+
+template <int T, int NKB, int NVB, int STAGES>
+cudaError_t launch_latent(const DecodeArgs &a, int slots, cudaStream_t st)
+{
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)a.row, (cuuint64_t)a.num_pages * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)a.row * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)T};
+    if (encode_tiled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.kv), dims, strides,
+                     box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(LatentSmem<T, NKB, STAGES>) + 1024;
+    auto kern = latent_tc_decode_kernel<T, NKB, NVB, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    kern<<<dim3(a.num_splits, slots, a.B), kThreads, smem, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Shapes the tensor-core latent kernel covers: MLA 512 + 64 (two value
+// halves), GLA with 256-wide latent heads + 64 rope, MLRA with 128-wide
+// branches + 64 rope; at most 128 query heads per MMA.
+int latent_tc_slots(const Problem &pr)
+{
+    if (!pr.latent || pr.dr != 64)
+        return 0;
+    if (pr.mlra)
+        return (pr.dn == 128 && pr.H <= kRows) ? pr.NU : 0;
+    if (pr.NU == 1)
+        return (pr.dn == 512 && pr.H <= kRows) ? 2 : 0;
+    return (pr.dn == 256 && pr.HPU <= kRows) ? pr.NU : 0;
+}
+
+cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_t st)
+{
+    const int slots = latent_tc_slots(pr);
+    if (pr.mlra)
+        return launch_latent<64, 3, 2, 4>(a, slots, st);
+    if (pr.NU == 1)
+        return launch_latent<32, 9, 4, 2>(a, slots, st);
+    return launch_latent<64, 5, 4, 3>(a, slots, st);
+}
+
+}  // namespace kvattn
