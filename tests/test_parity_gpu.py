@@ -1,10 +1,12 @@
 """GPU parity: the CUDA path (called through the C ABI) against the fp64 oracle.
 
-Tolerances (bf16 output): max |err| <= 2e-2 and relative L2 <= 5e-3 on out,
-|lse error| <= 1e-3.  fp32 output (the tiny MLA case) is also held to
-max |err| <= 1e-4: every product and sum there is fp32 over at most 512
-tokens of 80-wide dots, so the error is a few fp32 ulps of O(1) values times
-the accumulation depth.
+Tolerances (every case): max |err| <= 2e-2 and relative L2 <= 5e-3 on out,
+|lse error| <= 1e-3.  fp32 output computed by the generic CUDA-core kernel
+(the tiny MLA case) is also held to max |err| <= 1e-4: every product and sum
+there is fp32 over at most 512 tokens of 80-wide dots, so the error is a few
+fp32 ulps of O(1) values times the accumulation depth.  The tensor-core paths
+round the softmax weights to bf16 before P.V (relative error up to 2^-9 per
+weight), so fp32 output from them gets only the common tolerances.
 """
 
 import numpy as np
@@ -42,6 +44,15 @@ def check(out, lse, ref_out, ref_lse, fp32=False, what=""):
     assert dl.max() <= TOL_LSE, f"{what}: lse err {dl.max():.3e}"
 
 
+def kernel_of(name_or_shape):
+    """Name of the decode kernel the library plans for a workload shape."""
+    from shared_kv_caches_b200 import kvattn as K
+    s = name_or_shape
+    lo, hi = s.ctx
+    p = K.params_for(s, (hi + 63) // 64, 1024, hi)
+    return K.KERNEL_NAMES[K.kvattn_get_plan(s.variant_id, p).kernel]
+
+
 def run_gpu(inputs, dev, num_splits=0, max_seq_len=None):
     import torch
     from shared_kv_caches_b200.device import DeviceProblem
@@ -70,8 +81,9 @@ def test_parity_small(dev, oracle_mod, name):
     shape, lens = SMALL[name]
     x = W.make_inputs(shape, seed=0, seq_lens=lens)
     ref_out, ref_lse = oracle_mod.decode(x)
-    _, out, lse = run_gpu(x, dev)
-    check(out, lse, ref_out, ref_lse, fp32=shape.out_dtype == "fp32", what=name)
+    p, out, lse = run_gpu(x, dev)
+    tight = shape.out_dtype == "fp32" and p.plan_kernel_name() == "generic"
+    check(out, lse, ref_out, ref_lse, fp32=tight, what=name)
 
 
 SWEEP_LENS = [1, 2, 63, 64, 65, 127, 128, 4097]
@@ -128,12 +140,22 @@ def test_parity_full_size_sampled(dev, oracle_mod, name):
     check(g_out, g_lse, ref_out, ref_lse, what=name)
 
 
+def test_benchmark_shapes_use_the_specialised_kernels(dev):
+    """The benchmark shapes run on their specialised kernels, not the generic one."""
+    assert kernel_of(W.WORKLOADS["gqa"]) == "gqa"
+    assert kernel_of(W.WORKLOADS["mfa"]) == "mqa_tc"
+    for n in ("mla", "gla", "mlra_128k", "mlra_1m", "mlra_b8_128k"):
+        assert kernel_of(W.WORKLOADS[n]) == "latent_tc", n
+    assert kernel_of(W.WORKLOADS["tiny_mla"]) == "generic"
+
+
 def test_tiny_config_exact_shape(dev, oracle_mod):
     """The tiny contiguous MLA problem, whole, fp32 output."""
     x = W.make_inputs(W.WORKLOADS["tiny_mla"], seed=0)
     ref_out, ref_lse = oracle_mod.decode(x)
     p, out, lse = run_gpu(x, dev)
     assert p.out.dtype.is_floating_point and p.out.element_size() == 4
+    assert p.plan_kernel_name() == "generic"
     check(out, lse, ref_out, ref_lse, fp32=True, what="tiny")
 
 
