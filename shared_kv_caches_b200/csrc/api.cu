@@ -143,8 +143,18 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         base = (long long)pr.B * pr.NU * pl->head_chunks;
         splits = choose_splits(forced_splits, base, max_pages, 2LL * kNumSMs, 1);
     }
-    const int pps = (max_pages + splits - 1) / splits;
+    int pps = (max_pages + splits - 1) / splits;
+    if (pl->pub.kernel == KVATTN_KERNEL_LATENT_TC) {
+        // whole tiles per part, and no more pages than the kernel's page table holds
+        const int m = latent_tc_page_multiple(pr);
+        const int cap = latent_tc_max_pages_per_split();
+        pps = (pps + m - 1) / m * m;
+        if (pps > cap)
+            pps = cap;
+    }
     splits = (max_pages + pps - 1) / pps;
+    if (splits > kMaxSplits)
+        return KVATTN_ERR_UNSUPPORTED;
     pl->pub.num_splits = splits;
     pl->pub.pages_per_split = pps;
     pl->pub.ctas = (int32_t)(base * splits);

@@ -16,7 +16,7 @@ namespace kvattn {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 512;
 
 __device__ float block_max(float v, float *red)
 {
@@ -50,12 +50,14 @@ __device__ float block_sum(float v, float *red)
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 {
-    extern __shared__ float w_s[];     // [R][S] merge weights
+    extern __shared__ float smem[];    // [R][S] merge weights, then [G][Dv] partial sums
     __shared__ float red[32];
     const int h = blockIdx.x, b = blockIdx.y;
     const int R = a.mlra ? a.NU : 1;
     const int S = a.num_splits;
     const int tid = threadIdx.x;
+    float *w_s = smem;
+    float *acc_s = smem + ((R * S + 3) & ~3);
 
     for (int r = 0; r < R; ++r) {
         const int hu = a.mlra ? h * R + r : h;
@@ -79,22 +81,43 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
     }
     __syncthreads();
 
-    for (int d = tid; d < a.Dv; d += kThreads) {
-        float acc = 0.f;
-        for (int r = 0; r < R; ++r) {
-            const int hu = a.mlra ? h * R + r : h;
-            const float *po = a.po + ((size_t)b * S * a.HU + hu) * a.Dv + d;
-            for (int s = 0; s < S; ++s) {
-                const float w = w_s[r * S + s];
-                if (w != 0.f)
-                    acc = fmaf(w, po[(size_t)s * a.HU * a.Dv], acc);
+    // G groups of Dv threads split the (branch, part) rows; each thread owns
+    // one value column and keeps four row loads in flight (Dv <= 512)
+    const int G = kThreads / a.Dv;
+    const int g = tid / a.Dv, d = tid % a.Dv;
+    const int rows = R * S;
+    float acc = 0.f;
+    if (g < G) {
+        int k = g;
+        for (; k + 3 * G < rows; k += 4 * G) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int kk = k + u * G, r = kk / S, s = kk % S;
+                const int hu = a.mlra ? h * R + r : h;
+                v[u] = a.po[(((size_t)b * S + s) * a.HU + hu) * a.Dv + d];
             }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                acc = fmaf(w_s[k + u * G], v[u], acc);
         }
-        const size_t o = ((size_t)b * a.H + h) * a.Dv + d;
+        for (; k < rows; k += G) {
+            const int r = k / S, s = k % S;
+            const int hu = a.mlra ? h * R + r : h;
+            acc = fmaf(w_s[k], a.po[(((size_t)b * S + s) * a.HU + hu) * a.Dv + d], acc);
+        }
+        acc_s[g * a.Dv + d] = acc;
+    }
+    __syncthreads();
+    if (tid < a.Dv) {
+        float sum = 0.f;
+        for (int gg = 0; gg < G; ++gg)
+            sum += acc_s[gg * a.Dv + tid];
+        const size_t o = ((size_t)b * a.H + h) * a.Dv + tid;
         if (a.out_fp32)
-            static_cast<float *>(a.out)[o] = acc;
+            static_cast<float *>(a.out)[o] = sum;
         else
-            static_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(acc);
+            static_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(sum);
     }
 }
 
@@ -103,7 +126,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st)
 {
     const int R = a.mlra ? a.NU : 1;
-    const size_t smem = (size_t)R * a.num_splits * sizeof(float);
+    const int G = kThreads / a.Dv;
+    const size_t smem = ((size_t)((R * a.num_splits + 3) & ~3) + (size_t)G * a.Dv) * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);

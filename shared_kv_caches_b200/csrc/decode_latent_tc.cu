@@ -14,10 +14,17 @@
 // branch for MLRA.  Key columns of the slot are [latent slice | shared rope
 // key], each a 64-column box of the page row.
 //
+// The query rows are the MMA's A operand for every tile.  Their first NQT
+// 64-column chunks sit in TMEM (an A operand in TMEM costs no shared-memory
+// bandwidth; with a narrow score tile the re-read of a 128-row A from shared
+// memory would otherwise bound the MMA), the rest in shared memory.  TMEM
+// columns: two score / probability buffers of T, the output slice, the Q
+// chunks (MLRA 256 + 128 + 96, MLA and GLA 128 + 256 + 128).
+//
 // Warp roles (192 threads):
 //   warp 0     TMEM allocation; one thread streams each tile's key boxes into
 //              a STAGES-deep shared-memory ring with 2-D TMA loads (128-byte
-//              swizzle, completion on kv_full)
+//              swizzle, completion on kv_full; a 128-token tile is two pages)
 //   warp 1     one thread issues S_j = Q K_j^T into one of two TMEM score
 //              buffers, then P_{j-1} V_{j-1} into the TMEM output; the warp
 //              zeroes the rows of a tile past the context first (0 * NaN
@@ -46,12 +53,17 @@ constexpr int kQChunkBytes = kRows * 128;  // 128 rows x 64 bf16, 128-byte swizz
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
-template <int T, int NKB, int STAGES>
+constexpr int kMaxSplitPages = 1024;       // pages per part the page-validity table holds
+constexpr int kPageBoxBytes = kPage * 128; // one page x 64 columns
+
+template <int T, int NKB, int STAGES, int NQT>
 struct LatentSmem {
     static constexpr int kBoxBytes = T * 128;
     static constexpr int kStageBytes = NKB * kBoxBytes;
-    unsigned char q[NKB][kQChunkBytes];
+    static constexpr int kQSmem = NKB - NQT > 0 ? NKB - NQT : 1;
+    unsigned char q[kQSmem][kQChunkBytes];    // Q chunks NQT..NKB-1 (K-major, 128-byte swizzle)
     unsigned char kv[STAGES][kStageBytes];
+    uint8_t pvalid[kMaxSplitPages];
     uint64_t kv_full[STAGES];
     uint64_t kv_empty[STAGES];
     uint64_t s_full[2];
@@ -62,33 +74,41 @@ struct LatentSmem {
     uint32_t tmem_base;
 };
 
-struct TileInfo {
-    long long page;
-    int off;    // token offset of the tile inside its page
-    int ntok;   // context tokens in the tile (0 if the page id is bad)
-};
-
-template <int T>
-__device__ __forceinline__ TileInfo tile_info(const DecodeArgs &a, int b, int L, int p0, int j)
+__device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
 {
-    TileInfo ti;
-    const int tok0 = p0 * kPage + j * T;
-    const int pi = tok0 / kPage;
-    ti.off = tok0 % kPage;
-    ti.page = a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
-    const bool ok = ti.page >= 0 && ti.page < a.num_pages;
-    ti.ntok = ok ? min(T, L - tok0) : 0;
-    return ti;
+    return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
 }
 
-template <int T, int NKB, int NVB, int STAGES>
+__device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
+{
+    return page >= 0 && page < a.num_pages;
+}
+
+// Context tokens in tile j of the part starting at page p0 (0 if one of its
+// pages has a bad id); pvalid holds one flag per page of the part.
+template <int T>
+__device__ __forceinline__ int tile_ntok(const uint8_t *pvalid, int L, int p0, int j)
+{
+    const int tok0 = p0 * kPage + j * T;
+    const int ntok = min(T, L - tok0);
+    bool ok = true;
+#pragma unroll
+    for (int sub = 0; sub < T / kPage; ++sub)
+        if (sub * kPage < ntok)
+            ok = ok && pvalid[j * (T / kPage) + sub];
+    return ok ? ntok : 0;
+}
+
+template <int T, int NKB, int NVB, int STAGES, int NQT>
 __global__ void __launch_bounds__(kThreads, 1)
     latent_tc_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a)
 {
-    using Smem = LatentSmem<T, NKB, STAGES>;
+    using Smem = LatentSmem<T, NKB, STAGES, NQT>;
     constexpr int kBoxBytes = Smem::kBoxBytes;
     constexpr int kDvSlot = NVB * 64;                            // value columns of this CTA
-    constexpr uint32_t kTmemCols = (2 * T + kDvSlot) <= 256 ? 256 : 512;
+    constexpr int kColsUsed = 2 * T + kDvSlot + NQT * 32;
+    static_assert(kColsUsed <= 512, "TMEM budget");
+    constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
     constexpr uint32_t kIdescS = idesc_bf16_f32(kRows, T, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kRows, kDvSlot, false, true);
 
@@ -132,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tbase = S.tmem_base;
     const uint32_t tS = tbase;                 // 2 score / probability buffers of T columns
     const uint32_t tO = tbase + 2 * T;         // kDvSlot output columns
+    const uint32_t tQ = tO + kDvSlot;          // NQT query chunks of 32 columns (bf16 pairs)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA
@@ -145,20 +166,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
                     break;
                 }
-                const TileInfo ti = tile_info<T>(a, b, L, p0, j);
                 issued = j + 1;
-                if (ti.ntok == 0) {
-                    if (slot == 0 && ti.off == 0)
+                const int tok0 = p0 * kPage + j * T;
+                const int ntok = min(T, L - tok0);
+                const int nsub = (ntok + kPage - 1) / kPage;     // pages of this tile holding context
+                long long pages[T / kPage];
+                bool ok = true;
+#pragma unroll
+                for (int sub = 0; sub < T / kPage; ++sub) {
+                    pages[sub] = sub < nsub ? page_id(a, b, tok0 / kPage + sub) : 0;
+                    if (sub < nsub && !page_ok(a, pages[sub]))
+                        ok = false;
+                }
+                if (!ok) {
+                    if (slot == 0)
                         raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);
                     mbar_arrive(&S.kv_full[st]);
                     continue;
                 }
-                mbar_arrive_expect_tx(&S.kv_full[st], Smem::kStageBytes);
-                const int y = (int)(ti.page * kPage) + ti.off;
+                mbar_arrive_expect_tx(&S.kv_full[st], (uint32_t)(nsub * NKB * kPageBoxBytes));
+                const int off = tok0 % kPage;
 #pragma unroll
-                for (int i = 0; i < NKB; ++i) {
-                    const int col = i < dn_boxes ? unit_col0 + 64 * i : a.NU * a.dn + 64 * (i - dn_boxes);
-                    tma_load_2d(S.kv[st] + i * kBoxBytes, &kv_map, col, y, &S.kv_full[st]);
+                for (int sub = 0; sub < T / kPage; ++sub) {
+                    if (sub >= nsub)
+                        break;
+                    const int y = (int)(pages[sub] * kPage) + off;
+#pragma unroll
+                    for (int i = 0; i < NKB; ++i) {
+                        const int col = i < dn_boxes ? unit_col0 + 64 * i : a.NU * a.dn + 64 * (i - dn_boxes);
+                        tma_load_2d(S.kv[st] + i * kBoxBytes + sub * kPageBoxBytes, &kv_map, col, y, &S.kv_full[st]);
+                    }
                 }
             }
             // every copy this thread started has landed before the CTA can exit
@@ -198,13 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            const TileInfo ti = tile_info<T>(a, b, L, p0, j);
-            if (ti.ntok < T) {
+            const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
+            if (ntok < T) {
                 // zero the rows past the context in every key box of the stage
-                const int rows = T - ti.ntok;
+                const int rows = T - ntok;
                 for (int idx = lane; idx < rows * NKB * 8; idx += 32) {
                     const int box = idx / (rows * 8), rem = idx % (rows * 8);
-                    const int row = ti.ntok + rem / 8, piece = rem % 8;
+                    const int row = ntok + rem / 8, piece = rem % 8;
                     *reinterpret_cast<uint4 *>(S.kv[st] + box * kBoxBytes + row * 128 + piece * 16) =
                         make_uint4(0, 0, 0, 0);
                 }
@@ -218,9 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < NKB; ++kb) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t qd = smem_desc(qbase + kb * kQChunkBytes + k * 32, 16, 1024, 2);
                         const uint64_t kd = smem_desc(kbase + kb * kBoxBytes + k * 32, 16, 1024, 2);
-                        umma_ss(tS + (j & 1) * T, qd, kd, kIdescS, (kb | k) ? 1u : 0u);
+                        if (kb < NQT) {
+                            umma_ts(tS + (j & 1) * T, tQ + kb * 32 + k * 8, kd, kIdescS, (kb | k) ? 1u : 0u);
+                        } else {
+                            const uint64_t qd = smem_desc(qbase + (kb - NQT) * kQChunkBytes + k * 32, 16, 1024, 2);
+                            umma_ss(tS + (j & 1) * T, qd, kd, kIdescS, (kb | k) ? 1u : 0u);
+                        }
                     }
                 }
                 umma_commit(&S.s_full[j & 1]);
@@ -249,7 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const int rows_used = a.mlra || mla ? a.H : a.HPU;     // GLA: the group's heads
         {
-            // Q row h of this slot: [latent query slice | rope query], swizzled
+            // validity of every page of this part (read by the MMA warp and here)
+            const int npg = min(a.pages_per_split, max(0, (L + kPage - 1) / kPage - p0));
+            for (int i = threadIdx.x - 64; i < npg; i += kSoftmaxThreads)
+                S.pvalid[i] = page_ok(a, page_id(a, b, p0 + i)) ? 1 : 0;
+            // Q row h of this slot: [latent query slice | rope query]; chunks
+            // below NQT go to TMEM (bf16 pairs), the rest to shared memory
             const __nv_bfloat16 *qn = nullptr, *qr = nullptr;
             if (h < rows_used) {
                 size_t row;
@@ -264,16 +310,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll 1
             for (int kb = 0; kb < NKB; ++kb) {
+                const __nv_bfloat16 *src = nullptr;
+                if (qn)
+                    src = kb < dn_boxes ? qn + 64 * kb : qr + 64 * (kb - dn_boxes);
+                if (kb < NQT) {
+                    uint32_t r[32];
 #pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (qn)
-                        v = kb < dn_boxes ? *reinterpret_cast<const uint4 *>(qn + 64 * kb + 8 * p)
-                                          : *reinterpret_cast<const uint4 *>(qr + 64 * (kb - dn_boxes) + 8 * p);
-                    *reinterpret_cast<uint4 *>(&S.q[kb][h * 128 + ((p ^ (h & 7)) << 4)]) = v;
+                    for (int p = 0; p < 8; ++p) {
+                        const uint4 v = src ? *reinterpret_cast<const uint4 *>(src + 8 * p) : make_uint4(0, 0, 0, 0);
+                        r[4 * p] = v.x;
+                        r[4 * p + 1] = v.y;
+                        r[4 * p + 2] = v.z;
+                        r[4 * p + 3] = v.w;
+                    }
+                    tmem_st32(tQ + lane_addr + kb * 32, r);
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint4 v = src ? *reinterpret_cast<const uint4 *>(src + 8 * p) : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(&S.q[kb - NQT][h * 128 + ((p ^ (h & 7)) << 4)]) = v;
+                    }
                 }
             }
             fence_proxy_async_smem();
+            named_sync(1, kSoftmaxThreads);      // page table complete before any role reads it
+            tc_fence_before();
             mbar_arrive(&S.q_ready);
         }
 
@@ -296,11 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         s[32 * c + i] = __uint_as_float(r[i]);
                 }
             }
-            const TileInfo ti = tile_info<T>(a, b, L, p0, j);
+            const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
             float mt = -INFINITY;
 #pragma unroll
             for (int i = 0; i < T; ++i) {
-                s[i] = i < ti.ntok ? s[i] * a.scale_log2 : -INFINITY;
+                s[i] = i < ntok ? s[i] * a.scale_log2 : -INFINITY;
                 mt = fmaxf(mt, s[i]);
             }
             float alpha = 1.f;
@@ -399,18 +460,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tbase, kTmemCols);
 }
 
-template <int T, int NKB, int NVB, int STAGES>
+template <int T, int NKB, int NVB, int STAGES, int NQT>
 cudaError_t launch_latent(const DecodeArgs &a, int slots, cudaStream_t st)
 {
     CUtensorMap map;
     const cuuint64_t dims[2] = {(cuuint64_t)a.row, (cuuint64_t)a.num_pages * kPage};
     const cuuint64_t strides[1] = {(cuuint64_t)a.row * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)T};
+    const cuuint32_t box[2] = {64, (cuuint32_t)(T < kPage ? T : kPage)};
     if (encode_tiled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.kv), dims, strides,
                      box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(LatentSmem<T, NKB, STAGES>) + 1024;
-    auto kern = latent_tc_decode_kernel<T, NKB, NVB, STAGES>;
+    const size_t smem = sizeof(LatentSmem<T, NKB, STAGES, NQT>) + 1024;
+    auto kern = latent_tc_decode_kernel<T, NKB, NVB, STAGES, NQT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -423,6 +484,10 @@ cudaError_t launch_latent(const DecodeArgs &a, int slots, cudaStream_t st)
 // Shapes the tensor-core latent kernel covers: MLA 512 + 64 (two value
 // halves), GLA with 256-wide latent heads + 64 rope, MLRA with 128-wide
 // branches + 64 rope; at most 128 query heads per MMA.
+// Pages per part must be a whole number of tiles and fit the validity table.
+int latent_tc_page_multiple(const Problem &pr) { return pr.mlra ? 2 : 1; }
+int latent_tc_max_pages_per_split() { return kMaxSplitPages; }
+
 int latent_tc_slots(const Problem &pr)
 {
     if (!pr.latent || pr.dr != 64)
@@ -438,10 +503,10 @@ cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_
 {
     const int slots = latent_tc_slots(pr);
     if (pr.mlra)
-        return launch_latent<64, 3, 2, 4>(a, slots, st);
+        return launch_latent<128, 3, 2, 4, 3>(a, slots, st);
     if (pr.NU == 1)
-        return launch_latent<32, 9, 4, 2>(a, slots, st);
-    return launch_latent<64, 5, 4, 3>(a, slots, st);
+        return launch_latent<64, 9, 4, 2, 4>(a, slots, st);
+    return launch_latent<64, 5, 4, 4, 4>(a, slots, st);
 }
 
 }  // namespace kvattn
