@@ -118,7 +118,10 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunk = 128;
         pl->head_chunks = tc_slots;
         base = (long long)pr.B * tc_slots;
-        splits = choose_splits(forced_splits, base, max_pages, 4LL * kNumSMs, pr.mlra ? 16 : 64);
+        // one CTA per SM: one wave when the batch is small (long parts, little
+        // partial-output traffic), several waves to even out ragged batches
+        const long long waves = base >= kNumSMs / 2 ? 4 : 1;
+        splits = choose_splits(forced_splits, base, max_pages, waves * kNumSMs, pr.mlra ? 16 : 64);
     } else if (gqa_supported(pr)) {
         pl->pub.kernel = KVATTN_KERNEL_GQA;
         pl->head_chunk = 4;

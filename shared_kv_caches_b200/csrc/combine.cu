@@ -16,108 +16,105 @@ namespace kvattn {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 128;
 
-__device__ float block_max(float v, float *red)
-{
-    for (int o = 16; o; o >>= 1)
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
-    if (lane == 0)
-        red[w] = v;
-    __syncthreads();
-    float r = -INFINITY;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i)
-        r = fmaxf(r, red[i]);
-    return r;
-}
-
-__device__ float block_sum(float v, float *red)
-{
-    for (int o = 16; o; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
-    if (lane == 0)
-        red[w] = v;
-    __syncthreads();
-    float r = 0.f;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i)
-        r += red[i];
-    return r;
-}
-
+// One block per (head, sequence).  Warp 0 turns the parts' lse values into
+// merge weights (per branch for MLRA); then G groups of Dv/4 threads split
+// the (branch, part) rows, each thread owning four value columns (float4) and
+// keeping four row loads in flight; the groups' sums meet in shared memory.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 {
-    extern __shared__ float smem[];    // [R][S] merge weights, then [G][Dv] partial sums
-    __shared__ float red[32];
+    extern __shared__ float4 smem4[];  // [G][Dv/4] partial sums, then [R][S] weights
     const int h = blockIdx.x, b = blockIdx.y;
     const int R = a.mlra ? a.NU : 1;
     const int S = a.num_splits;
-    const int tid = threadIdx.x;
-    float *w_s = smem;
-    float *acc_s = smem + ((R * S + 3) & ~3);
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int V4 = a.Dv / 4;
+    const int G = kThreads / V4;
+    float4 *acc_s = smem4;
+    float *w_s = reinterpret_cast<float *>(smem4 + G * V4);
 
-    for (int r = 0; r < R; ++r) {
-        const int hu = a.mlra ? h * R + r : h;
-        const float *pl = a.plse + (size_t)b * S * a.HU + hu;
-        float mx = -INFINITY;
-        for (int s = tid; s < S; s += kThreads)
-            mx = fmaxf(mx, pl[(size_t)s * a.HU]);
-        mx = block_max(mx, red);
-        float sum = 0.f;
-        for (int s = tid; s < S; s += kThreads) {
-            const float w = mx == -INFINITY ? 0.f : expf(pl[(size_t)s * a.HU] - mx);
-            w_s[r * S + s] = w;
-            sum += w;
+    if (tid < 32) {
+        for (int r = 0; r < R; ++r) {
+            const int hu = a.mlra ? h * R + r : h;
+            const float *pl = a.plse + (size_t)b * S * a.HU + hu;
+            float mx = -INFINITY;
+            for (int s = lane; s < S; s += 32)
+                mx = fmaxf(mx, pl[(size_t)s * a.HU]);
+            for (int o = 16; o; o >>= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            float sum = 0.f;
+            for (int s = lane; s < S; s += 32) {
+                const float w = mx == -INFINITY ? 0.f : expf(pl[(size_t)s * a.HU] - mx);
+                w_s[r * S + s] = w;
+                sum += w;
+            }
+            for (int o = 16; o; o >>= 1)
+                sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const float inv = sum > 0.f ? 1.f / sum : 0.f;
+            for (int s = lane; s < S; s += 32)
+                w_s[r * S + s] *= inv;
+            if (lane == 0 && a.lse)
+                a.lse[(size_t)b * a.HU + hu] = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + logf(sum);
         }
-        sum = block_sum(sum, red);
-        const float inv = sum > 0.f ? 1.f / sum : 0.f;
-        for (int s = tid; s < S; s += kThreads)
-            w_s[r * S + s] *= inv;
-        if (tid == 0 && a.lse)
-            a.lse[(size_t)b * a.HU + hu] = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + logf(sum);
     }
     __syncthreads();
 
-    // G groups of Dv threads split the (branch, part) rows; each thread owns
-    // one value column and keeps four row loads in flight (Dv <= 512)
-    const int G = kThreads / a.Dv;
-    const int g = tid / a.Dv, d = tid % a.Dv;
+    const int g = tid / V4, d4 = tid % V4;
     const int rows = R * S;
-    float acc = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (g < G) {
-        int k = g;
-        for (; k + 3 * G < rows; k += 4 * G) {
-            float v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int kk = k + u * G, r = kk / S, s = kk % S;
-                const int hu = a.mlra ? h * R + r : h;
-                v[u] = a.po[(((size_t)b * S + s) * a.HU + hu) * a.Dv + d];
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                acc = fmaf(w_s[k + u * G], v[u], acc);
-        }
-        for (; k < rows; k += G) {
+        auto row_ptr = [&](int k) {
             const int r = k / S, s = k % S;
             const int hu = a.mlra ? h * R + r : h;
-            acc = fmaf(w_s[k], a.po[(((size_t)b * S + s) * a.HU + hu) * a.Dv + d], acc);
+            return reinterpret_cast<const float4 *>(a.po + (((size_t)b * S + s) * a.HU + hu) * a.Dv) + d4;
+        };
+        int k = g;
+        for (; k + 3 * G < rows; k += 4 * G) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                v[u] = *row_ptr(k + u * G);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float w = w_s[k + u * G];
+                acc.x = fmaf(w, v[u].x, acc.x);
+                acc.y = fmaf(w, v[u].y, acc.y);
+                acc.z = fmaf(w, v[u].z, acc.z);
+                acc.w = fmaf(w, v[u].w, acc.w);
+            }
         }
-        acc_s[g * a.Dv + d] = acc;
+        for (; k < rows; k += G) {
+            const float4 v = *row_ptr(k);
+            const float w = w_s[k];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        acc_s[g * V4 + d4] = acc;
     }
     __syncthreads();
-    if (tid < a.Dv) {
-        float sum = 0.f;
-        for (int gg = 0; gg < G; ++gg)
-            sum += acc_s[gg * a.Dv + tid];
-        const size_t o = ((size_t)b * a.H + h) * a.Dv + tid;
-        if (a.out_fp32)
-            static_cast<float *>(a.out)[o] = sum;
-        else
-            static_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(sum);
+    if (tid < V4) {
+        float4 sum = acc_s[tid];
+        for (int gg = 1; gg < G; ++gg) {
+            const float4 v = acc_s[gg * V4 + tid];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+        }
+        const size_t o = ((size_t)b * a.H + h) * a.Dv + 4 * tid;
+        if (a.out_fp32) {
+            *reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o) = sum;
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+            uint2 packed;
+            packed.x = *reinterpret_cast<const uint32_t *>(&lo);
+            packed.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.out) + o) = packed;
+        }
     }
 }
 
@@ -126,8 +123,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st)
 {
     const int R = a.mlra ? a.NU : 1;
-    const int G = kThreads / a.Dv;
-    const size_t smem = ((size_t)((R * a.num_splits + 3) & ~3) + (size_t)G * a.Dv) * sizeof(float);
+    const int V4 = a.Dv / 4;
+    const int G = kThreads / V4;
+    const size_t smem = (size_t)G * V4 * sizeof(float4) + (size_t)R * a.num_splits * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);

@@ -348,22 +348,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             float s[T];
             {
-                uint32_t r[32];
+                uint32_t r[T];
+                if constexpr (T == 128)
+                    tmem_ld128(tS + lane_addr + sb * T, r);
+                else
+                    tmem_ld64(tS + lane_addr + sb * T, r);
 #pragma unroll
-                for (int c = 0; c < T / 32; ++c) {
-                    tmem_ld32(tS + lane_addr + sb * T + 32 * c, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        s[32 * c + i] = __uint_as_float(r[i]);
-                }
+                for (int i = 0; i < T; ++i)
+                    s[i] = __uint_as_float(r[i]);
             }
             const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
-            float mt = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < T; ++i) {
+            for (int i = 0; i < T; ++i)
                 s[i] = i < ntok ? s[i] * a.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, s[i]);
+            // tree reduction of the tile max (independent chains)
+            float mx8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                mx8[q] = s[q];
+#pragma unroll
+                for (int i = q + 8; i < T; i += 8)
+                    mx8[q] = fmaxf(mx8[q], s[i]);
             }
+            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref + kRescaleThreshold) {
@@ -374,19 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_ref = mt;
             }
             const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-            float ps = 0.f;
+            float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[T / 2];
 #pragma unroll
             for (int i = 0; i < T / 2; ++i) {
                 const float e0 = exp2f(s[2 * i] - m_use), e1 = exp2f(s[2 * i + 1] - m_use);
-                ps += e0 + e1;
+                ps8[i & 7] += e0 + e1;
                 const __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
                 pk[i] = *reinterpret_cast<const uint32_t *>(&v2);
             }
+            const float ps = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
             l = l * alpha + ps;
-#pragma unroll
-            for (int c = 0; c < T / 32; ++c)
-                tmem_st16(tS + lane_addr + sb * T + 16 * c, pk + 16 * c);
+            if constexpr (T == 128)
+                tmem_st64(tS + lane_addr + sb * T, pk);
+            else
+                tmem_st32(tS + lane_addr + sb * T, pk);
             // TMEM accesses are warp-wide: rescale the whole warp's rows when any needs it
             if (__any_sync(0xffffffffu, rescale)) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (j - 1) & 1));
@@ -432,19 +442,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t prow = ((size_t)b * a.num_splits + split) * a.HU + (valid ? hu : 0);
         float *dst = a.po + prow * a.dn + col0;
         const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-        uint32_t r[32];
+        uint32_t r[64];
 #pragma unroll 1
-        for (int c = 0; c < kDvSlot / 32; ++c) {
+        for (int c = 0; c < kDvSlot / 64; ++c) {
             if (have)
-                tmem_ld32(tO + lane_addr + 32 * c, r);
+                tmem_ld64(tO + lane_addr + 64 * c, r);
             if (valid) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
+                for (int i = 0; i < 64; i += 4) {
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (have)
                         v = make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
                                         __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
-                    *reinterpret_cast<float4 *>(dst + 32 * c + i) = v;
+                    *reinterpret_cast<float4 *>(dst + 64 * c + i) = v;
                 }
             }
         }

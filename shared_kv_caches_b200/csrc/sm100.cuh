@@ -218,6 +218,52 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+// 64 consecutive columns in one load, waited.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, "
+        "%38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, "
+        "%60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : KV_R8(0), KV_R8(8), KV_R8(16), KV_R8(24), KV_R8(32), KV_R8(40), KV_R8(48), KV_R8(56)
+        : "r"(taddr)
+        : "memory");
+}
+
+// 128 consecutive columns: two 64-column loads under one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, "
+        "%38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, "
+        "%60, %61, %62, %63}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, "
+        "%78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, "
+        "%100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, "
+        "%118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%129];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : KV_R8(0), KV_R8(8), KV_R8(16), KV_R8(24), KV_R8(32), KV_R8(40), KV_R8(48), KV_R8(56), KV_R8(64), KV_R8(72),
+          KV_R8(80), KV_R8(88), KV_R8(96), KV_R8(104), KV_R8(112), KV_R8(120)
+        : "r"(taddr), "r"(taddr + 64)
+        : "memory");
+}
+
+// 64 consecutive columns in one store, waited.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, "
+        "%37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, "
+        "%59, %60, %61, %62, %63, %64};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        KV_W8(0), KV_W8(8), KV_W8(16), KV_W8(24), KV_W8(32), KV_W8(40), KV_W8(48), KV_W8(56)
+        : "memory");
+}
+
 #undef KV_R8
 #undef KV_W8
 
