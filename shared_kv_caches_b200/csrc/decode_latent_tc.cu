@@ -29,10 +29,12 @@
 //              buffers, then P_{j-1} V_{j-1} into the TMEM output; the warp
 //              zeroes the rows of a tile past the context first (0 * NaN
 //              would poison the MMA)
-//   warps 2-5  one thread per head row: read S_j from TMEM, online softmax in
-//              fp32 (base 2) with a lazy rescale (the reference max moves
-//              only when a score exceeds it by more than 2^8, so O is
-//              rarely touched), write P_j as bf16 into the score buffer it
+//   warps 2-9  two threads per head row, each owning half of the tile's
+//              columns and half of O's: read S_j from TMEM, exchange the tile
+//              maximum with the partner thread through shared memory, online
+//              softmax in fp32 (base 2) with a lazy rescale (the reference
+//              max moves only when a score exceeds it by more than 2^8, so O
+//              is rarely touched), write P_j as bf16 into the score buffer it
 //              came from (the A operand of the P.V MMA), and at the end
 //              normalise O and write the part result and its lse.
 // Every wait is bounded; a wait that gives up sets an error bit and the CTA
@@ -47,7 +49,7 @@ namespace kvattn {
 namespace {
 
 constexpr int kRows = 128;                 // MMA M: query-head rows
-constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxThreads = 256;       // two warps per TMEM lane quarter
 constexpr int kThreads = 64 + kSoftmaxThreads;
 constexpr int kQChunkBytes = kRows * 128;  // 128 rows x 64 bf16, 128-byte swizzle
 constexpr float kLn2 = 0.69314718055994531f;
@@ -63,7 +65,8 @@ struct LatentSmem {
     static constexpr int kQSmem = NKB - NQT > 0 ? NKB - NQT : 1;
     unsigned char q[kQSmem][kQChunkBytes];    // Q chunks NQT..NKB-1 (K-major, 128-byte swizzle)
     unsigned char kv[STAGES][kStageBytes];
-    uint8_t pvalid[kMaxSplitPages];
+    float xmax[2][2][kRows];                  // [exchange parity][column half][row]
+    uint32_t pvalid[kMaxSplitPages / 32];     // one bit per page of the part
     uint64_t kv_full[STAGES];
     uint64_t kv_empty[STAGES];
     uint64_t s_full[2];
@@ -71,6 +74,7 @@ struct LatentSmem {
     uint64_t o_ready;
     uint64_t q_ready;
     uint64_t mma_done;
+    uint64_t xbar[4];                         // per lane quarter: the two threads of a row meet here
     uint32_t tmem_base;
 };
 
@@ -85,17 +89,19 @@ __device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
 }
 
 // Context tokens in tile j of the part starting at page p0 (0 if one of its
-// pages has a bad id); pvalid holds one flag per page of the part.
+// pages has a bad id); pvalid holds one bit per page of the part.
 template <int T>
-__device__ __forceinline__ int tile_ntok(const uint8_t *pvalid, int L, int p0, int j)
+__device__ __forceinline__ int tile_ntok(const uint32_t *pvalid, int L, int p0, int j)
 {
     const int tok0 = p0 * kPage + j * T;
     const int ntok = min(T, L - tok0);
     bool ok = true;
 #pragma unroll
-    for (int sub = 0; sub < T / kPage; ++sub)
+    for (int sub = 0; sub < T / kPage; ++sub) {
+        const int pg = j * (T / kPage) + sub;
         if (sub * kPage < ntok)
-            ok = ok && pvalid[j * (T / kPage) + sub];
+            ok = ok && ((pvalid[pg >> 5] >> (pg & 31)) & 1u);
+    }
     return ok ? ntok : 0;
 }
 
@@ -112,11 +118,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdescS = idesc_bf16_f32(kRows, T, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kRows, kDvSlot, false, true);
 
-    extern __shared__ unsigned char smem_raw[];
-    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
     const bool mla = !a.mlra && a.NU == 1;
+    if (smem_u32(smem_raw) & 1023u) {
+        // the 128-byte swizzle atoms need 1024-byte alignment; never expected
+        if (threadIdx.x == 0)
+            raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+        return;
+    }
     const int dn_boxes = a.dn / 64;
 
     int L = a.seq_lens[b];
@@ -142,6 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.o_ready, 1);
         mbar_init(&S.q_ready, kSoftmaxThreads);
         mbar_init(&S.mma_done, 1);
+        for (int q = 0; q < 4; ++q)
+            mbar_init(&S.xbar[q], 64);
         fence_mbar_init();
     }
     if (warp == 0)
@@ -285,17 +299,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
+        constexpr int TH = T / 2;                                // score columns per thread
+        constexpr int OH = kDvSlot / 2;                          // output columns per thread
+        const int sw = warp - 2;                                 // 0..7
         const int quarter = warp & 3;
-        const int h = quarter * 32 + lane;                      // head row = TMEM lane
+        const int half = sw >> 2;                                // column half
+        const int h = quarter * 32 + lane;                       // head row = TMEM lane
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const int rows_used = a.mlra || mla ? a.H : a.HPU;     // GLA: the group's heads
+        const int rows_used = a.mlra || mla ? a.H : a.HPU;      // GLA: the group's heads
         {
             // validity of every page of this part (read by the MMA warp and here)
             const int npg = min(a.pages_per_split, max(0, (L + kPage - 1) / kPage - p0));
-            for (int i = threadIdx.x - 64; i < npg; i += kSoftmaxThreads)
-                S.pvalid[i] = page_ok(a, page_id(a, b, p0 + i)) ? 1 : 0;
+            for (int w = threadIdx.x - 64; w < (npg + 31) / 32; w += kSoftmaxThreads) {
+                uint32_t bits = 0;
+                for (int i = 32 * w; i < min(npg, 32 * w + 32); ++i)
+                    bits |= (page_ok(a, page_id(a, b, p0 + i)) ? 1u : 0u) << (i & 31);
+                S.pvalid[w] = bits;
+            }
             // Q row h of this slot: [latent query slice | rope query]; chunks
-            // below NQT go to TMEM (bf16 pairs), the rest to shared memory
+            // below NQT go to TMEM (bf16 pairs), the rest to shared memory;
+            // the two threads of a row take alternate chunks
             const __nv_bfloat16 *qn = nullptr, *qr = nullptr;
             if (h < rows_used) {
                 size_t row;
@@ -309,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 qr = a.q_rope + row * a.dr;
             }
 #pragma unroll 1
-            for (int kb = 0; kb < NKB; ++kb) {
+            for (int kb = half; kb < NKB; kb += 2) {
                 const __nv_bfloat16 *src = nullptr;
                 if (qn)
                     src = kb < dn_boxes ? qn + 64 * kb : qr + 64 * (kb - dn_boxes);
@@ -338,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&S.q_ready);
         }
 
-        float m_ref = -INFINITY, l = 0.f;
+        float m_ref = -INFINITY, l = 0.f;       // l: this thread's half of the row sum
         bool ok = true;
         for (int j = 0; j < n; ++j) {
             const int sb = j & 1;
@@ -346,32 +369,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            float s[T];
+            const uint32_t s_addr = tS + lane_addr + sb * T + half * TH;
+            float s[TH];
             {
-                uint32_t r[T];
-                if constexpr (T == 128)
-                    tmem_ld128(tS + lane_addr + sb * T, r);
+                uint32_t r[TH];
+                if constexpr (TH == 64)
+                    tmem_ld64(s_addr, r);
                 else
-                    tmem_ld64(tS + lane_addr + sb * T, r);
+                    tmem_ld32(s_addr, r);
 #pragma unroll
-                for (int i = 0; i < T; ++i)
-                    s[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < TH; ++i)
+                    s[i] = __uint_as_float(r[i]) * a.scale_log2;
             }
             const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
+            if (ntok < T) {
 #pragma unroll
-            for (int i = 0; i < T; ++i)
-                s[i] = i < ntok ? s[i] * a.scale_log2 : -INFINITY;
-            // tree reduction of the tile max (independent chains)
+                for (int i = 0; i < TH; ++i)
+                    s[i] = half * TH + i < ntok ? s[i] : -INFINITY;
+            }
             float mx8[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 mx8[q] = s[q];
 #pragma unroll
-                for (int i = q + 8; i < T; i += 8)
+                for (int i = q + 8; i < TH; i += 8)
                     mx8[q] = fmaxf(mx8[q], s[i]);
             }
-            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            // the row max over both halves: swap through shared memory with the
+            // partner warp (bounded wait on the quarter's exchange barrier)
+            S.xmax[sb][half][h] = mt;
+            mbar_arrive(&S.xbar[quarter]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&S.xbar[quarter], j & 1));
+            if (!ok)
+                break;
+            mt = fmaxf(mt, S.xmax[sb][half ^ 1][h]);
+
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref + kRescaleThreshold) {
@@ -383,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
             float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[T / 2];
+            uint32_t pk[TH / 2];
 #pragma unroll
-            for (int i = 0; i < T / 2; ++i) {
+            for (int i = 0; i < TH / 2; ++i) {
                 const float e0 = exp2f(s[2 * i] - m_use), e1 = exp2f(s[2 * i + 1] - m_use);
                 ps8[i & 7] += e0 + e1;
                 const __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
@@ -393,11 +427,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float ps = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
             l = l * alpha + ps;
-            if constexpr (T == 128)
-                tmem_st64(tS + lane_addr + sb * T, pk);
+            // P (bf16 pairs) over this half's columns of the score buffer
+            const uint32_t p_addr = tS + lane_addr + sb * T + half * (TH / 2);
+            if constexpr (TH / 2 == 32)
+                tmem_st32(p_addr, pk);
             else
-                tmem_st32(tS + lane_addr + sb * T, pk);
-            // TMEM accesses are warp-wide: rescale the whole warp's rows when any needs it
+                tmem_st16(p_addr, pk);
+            // TMEM accesses are warp-wide: rescale the warp's rows when any needs it
             if (__any_sync(0xffffffffu, rescale)) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (j - 1) & 1));
                 if (!ok)
@@ -405,12 +441,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 uint32_t r[32];
 #pragma unroll 1
-                for (int c = 0; c < kDvSlot / 32; ++c) {
-                    tmem_ld32(tO + lane_addr + 32 * c, r);
+                for (int c = 0; c < OH / 32; ++c) {
+                    const uint32_t o_addr = tO + lane_addr + half * OH + 32 * c;
+                    tmem_ld32(o_addr, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(tO + lane_addr + 32 * c, r);
+                    tmem_st32(o_addr, r);
                 }
             }
             tc_fence_before();
@@ -419,7 +456,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok && lane == 0)
             raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
 
-        // part result: O / l and lse for this row
+        // part result: O / l and lse for this row (l = sum of both halves,
+        // swapped in the exchange slot after the last tile's)
+        if (ok) {
+            S.xmax[n & 1][half][h] = l;
+            mbar_arrive(&S.xbar[quarter]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&S.xbar[quarter], n & 1));
+            if (ok)
+                l += S.xmax[n & 1][half ^ 1][h];
+            else if (lane == 0)
+                raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+        }
         bool have = false;
         if (ok && n > 0) {
             have = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (n - 1) & 1));
@@ -440,13 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             col0 = 0;
         }
         const size_t prow = ((size_t)b * a.num_splits + split) * a.HU + (valid ? hu : 0);
-        float *dst = a.po + prow * a.dn + col0;
+        float *dst = a.po + prow * a.dn + col0 + half * OH;
         const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
         uint32_t r[64];
 #pragma unroll 1
-        for (int c = 0; c < kDvSlot / 64; ++c) {
+        for (int c = 0; c < OH / 64; ++c) {
             if (have)
-                tmem_ld64(tO + lane_addr + 64 * c, r);
+                tmem_ld64(tO + lane_addr + half * OH + 64 * c, r);
             if (valid) {
 #pragma unroll
                 for (int i = 0; i < 64; i += 4) {
@@ -458,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        if (valid && (!mla || slot == 0))
+        if (valid && half == 0 && (!mla || slot == 0))
             a.plse[prow] = (have && l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
     }
     __syncwarp();
@@ -480,7 +527,7 @@ cudaError_t launch_latent(const DecodeArgs &a, int slots, cudaStream_t st)
     if (encode_tiled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.kv), dims, strides,
                      box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(LatentSmem<T, NKB, STAGES, NQT>) + 1024;
+    const size_t smem = sizeof(LatentSmem<T, NKB, STAGES, NQT>);
     auto kern = latent_tc_decode_kernel<T, NKB, NVB, STAGES, NQT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
