@@ -118,10 +118,21 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunk = 128;
         pl->head_chunks = tc_slots;
         base = (long long)pr.B * tc_slots;
-        // one CTA per SM: one wave when the batch is small (long parts, little
-        // partial-output traffic), several waves to even out ragged batches
-        const long long waves = base >= kNumSMs / 2 ? 4 : 1;
-        splits = choose_splits(forced_splits, base, max_pages, waves * kNumSMs, pr.mlra ? 16 : 64);
+        // one CTA per SM: for small batches the fewest waves that keep >= 90% of
+        // the SMs busy (long parts, little partial-output traffic); several
+        // waves to even out ragged large batches
+        long long target = 4LL * kNumSMs;
+        if (base < kNumSMs / 2) {
+            for (long long k = 1; k <= 4; ++k) {
+                const long long sp = (k * kNumSMs) / base;
+                const long long ctas = sp * base;
+                const long long waves = (ctas + kNumSMs - 1) / kNumSMs;
+                target = ctas;
+                if (sp >= 1 && ctas * 10 >= waves * kNumSMs * 9)
+                    break;
+            }
+        }
+        splits = choose_splits(forced_splits, base, max_pages, target, pr.mlra ? 16 : 64);
     } else if (gqa_supported(pr)) {
         pl->pub.kernel = KVATTN_KERNEL_GQA;
         pl->head_chunk = 4;

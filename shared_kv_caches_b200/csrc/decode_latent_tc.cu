@@ -56,7 +56,6 @@ constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
 constexpr int kMaxSplitPages = 1024;       // pages per part the page-validity table holds
-constexpr int kPageBoxBytes = kPage * 128; // one page x 64 columns
 
 template <int T, int NKB, int STAGES, int NQT>
 struct LatentSmem {
@@ -93,12 +92,13 @@ __device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
 template <int T>
 __device__ __forceinline__ int tile_ntok(const uint32_t *pvalid, int L, int p0, int j)
 {
+    constexpr int kSubs = T >= kPage ? T / kPage : 1;     // pages a tile spans
     const int tok0 = p0 * kPage + j * T;
     const int ntok = min(T, L - tok0);
     bool ok = true;
 #pragma unroll
-    for (int sub = 0; sub < T / kPage; ++sub) {
-        const int pg = j * (T / kPage) + sub;
+    for (int sub = 0; sub < kSubs; ++sub) {
+        const int pg = (j * T) / kPage + sub;
         if (sub * kPage < ntok)
             ok = ok && ((pvalid[pg >> 5] >> (pg & 31)) & 1u);
     }
@@ -181,13 +181,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 issued = j + 1;
+                constexpr int kSubs = T >= kPage ? T / kPage : 1;   // pages a tile spans
+                constexpr int kSubRows = T >= kPage ? kPage : T;    // rows per TMA box
                 const int tok0 = p0 * kPage + j * T;
                 const int ntok = min(T, L - tok0);
-                const int nsub = (ntok + kPage - 1) / kPage;     // pages of this tile holding context
-                long long pages[T / kPage];
+                const int nsub = (ntok + kSubRows - 1) / kSubRows;  // boxes of this tile holding context
+                long long pages[kSubs];
                 bool ok = true;
 #pragma unroll
-                for (int sub = 0; sub < T / kPage; ++sub) {
+                for (int sub = 0; sub < kSubs; ++sub) {
                     pages[sub] = sub < nsub ? page_id(a, b, tok0 / kPage + sub) : 0;
                     if (sub < nsub && !page_ok(a, pages[sub]))
                         ok = false;
@@ -198,17 +200,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&S.kv_full[st]);
                     continue;
                 }
-                mbar_arrive_expect_tx(&S.kv_full[st], (uint32_t)(nsub * NKB * kPageBoxBytes));
+                mbar_arrive_expect_tx(&S.kv_full[st], (uint32_t)(nsub * NKB * kSubRows * 128));
                 const int off = tok0 % kPage;
 #pragma unroll
-                for (int sub = 0; sub < T / kPage; ++sub) {
+                for (int sub = 0; sub < kSubs; ++sub) {
                     if (sub >= nsub)
                         break;
                     const int y = (int)(pages[sub] * kPage) + off;
 #pragma unroll
                     for (int i = 0; i < NKB; ++i) {
                         const int col = i < dn_boxes ? unit_col0 + 64 * i : a.NU * a.dn + 64 * (i - dn_boxes);
-                        tma_load_2d(S.kv[st] + i * kBoxBytes + sub * kPageBoxBytes, &kv_map, col, y, &S.kv_full[st]);
+                        tma_load_2d(S.kv[st] + i * kBoxBytes + sub * kSubRows * 128, &kv_map, col, y, &S.kv_full[st]);
                     }
                 }
             }
@@ -375,8 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t r[TH];
                 if constexpr (TH == 64)
                     tmem_ld64(s_addr, r);
-                else
+                else if constexpr (TH == 32)
                     tmem_ld32(s_addr, r);
+                else
+                    tmem_ld16(s_addr, r);
 #pragma unroll
                 for (int i = 0; i < TH; ++i)
                     s[i] = __uint_as_float(r[i]) * a.scale_log2;
@@ -431,8 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t p_addr = tS + lane_addr + sb * T + half * (TH / 2);
             if constexpr (TH / 2 == 32)
                 tmem_st32(p_addr, pk);
-            else
+            else if constexpr (TH / 2 == 16)
                 tmem_st16(p_addr, pk);
+            else
+                tmem_st8(p_addr, pk);
             // TMEM accesses are warp-wide: rescale the warp's rows when any needs it
             if (__any_sync(0xffffffffu, rescale)) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&S.o_ready, (j - 1) & 1));
@@ -562,7 +568,7 @@ cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_
     if (pr.mlra)
         return launch_latent<128, 3, 2, 4, 3>(a, slots, st);
     if (pr.NU == 1)
-        return launch_latent<64, 9, 4, 2, 4>(a, slots, st);
+        return launch_latent<32, 9, 4, 4, 5>(a, slots, st);
     return launch_latent<64, 5, 4, 4, 4>(a, slots, st);
 }
 

@@ -264,6 +264,14 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+                 "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+                 KV_W8(0)
+                 : "memory");
+}
+
 #undef KV_R8
 #undef KV_W8
 
