@@ -17,22 +17,24 @@ namespace kvattn {
 namespace {
 
 constexpr int kThreads = 128;
+constexpr int kColsPerBlock = 32;          // value columns a block merges (8 float4)
+constexpr int kV4 = kColsPerBlock / 4;
+constexpr int kGroups = kThreads / kV4;    // row groups per block
 
-// One block per (head, sequence).  Warp 0 turns the parts' lse values into
-// merge weights (per branch for MLRA); then G groups of Dv/4 threads split
-// the (branch, part) rows, each thread owning four value columns (float4) and
-// keeping four row loads in flight; the groups' sums meet in shared memory.
+// One block per (head, sequence, 32-column chunk of the value).  Warp 0 turns
+// the parts' lse values into merge weights (per branch for MLRA; every block
+// of a head recomputes them, which is cheap); then 16 groups of 8 threads
+// split the (branch, part) rows, each thread owning four value columns
+// (float4) with four row loads in flight; the groups meet in shared memory.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 {
-    extern __shared__ float4 smem4[];  // [G][Dv/4] partial sums, then [R][S] weights
+    extern __shared__ float w_s[];     // [R][S] merge weights
+    __shared__ float4 acc_s[kGroups][kV4];
     const int h = blockIdx.x, b = blockIdx.y;
+    const int c0 = blockIdx.z * kColsPerBlock;
     const int R = a.mlra ? a.NU : 1;
     const int S = a.num_splits;
     const int tid = threadIdx.x, lane = tid & 31;
-    const int V4 = a.Dv / 4;
-    const int G = kThreads / V4;
-    float4 *acc_s = smem4;
-    float *w_s = reinterpret_cast<float *>(smem4 + G * V4);
 
     if (tid < 32) {
         for (int r = 0; r < R; ++r) {
@@ -54,37 +56,39 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
             const float inv = sum > 0.f ? 1.f / sum : 0.f;
             for (int s = lane; s < S; s += 32)
                 w_s[r * S + s] *= inv;
-            if (lane == 0 && a.lse)
+            if (lane == 0 && a.lse && blockIdx.z == 0)
                 a.lse[(size_t)b * a.HU + hu] = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + logf(sum);
         }
     }
     __syncthreads();
 
-    const int g = tid / V4, d4 = tid % V4;
+    const int g = tid / kV4, q4 = tid % kV4;
+    const int col = c0 + 4 * q4;
+    const bool on = col < a.Dv;
     const int rows = R * S;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (g < G) {
+    if (on) {
         auto row_ptr = [&](int k) {
             const int r = k / S, s = k % S;
             const int hu = a.mlra ? h * R + r : h;
-            return reinterpret_cast<const float4 *>(a.po + (((size_t)b * S + s) * a.HU + hu) * a.Dv) + d4;
+            return reinterpret_cast<const float4 *>(a.po + (((size_t)b * S + s) * a.HU + hu) * a.Dv + col);
         };
         int k = g;
-        for (; k + 3 * G < rows; k += 4 * G) {
+        for (; k + 3 * kGroups < rows; k += 4 * kGroups) {
             float4 v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                v[u] = *row_ptr(k + u * G);
+                v[u] = *row_ptr(k + u * kGroups);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float w = w_s[k + u * G];
+                const float w = w_s[k + u * kGroups];
                 acc.x = fmaf(w, v[u].x, acc.x);
                 acc.y = fmaf(w, v[u].y, acc.y);
                 acc.z = fmaf(w, v[u].z, acc.z);
                 acc.w = fmaf(w, v[u].w, acc.w);
             }
         }
-        for (; k < rows; k += G) {
+        for (; k < rows; k += kGroups) {
             const float4 v = *row_ptr(k);
             const float w = w_s[k];
             acc.x = fmaf(w, v.x, acc.x);
@@ -92,19 +96,19 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
             acc.z = fmaf(w, v.z, acc.z);
             acc.w = fmaf(w, v.w, acc.w);
         }
-        acc_s[g * V4 + d4] = acc;
     }
+    acc_s[g][q4] = acc;
     __syncthreads();
-    if (tid < V4) {
-        float4 sum = acc_s[tid];
-        for (int gg = 1; gg < G; ++gg) {
-            const float4 v = acc_s[gg * V4 + tid];
+    if (tid < kV4 && on) {
+        float4 sum = acc_s[0][tid];
+        for (int gg = 1; gg < kGroups; ++gg) {
+            const float4 v = acc_s[gg][tid];
             sum.x += v.x;
             sum.y += v.y;
             sum.z += v.z;
             sum.w += v.w;
         }
-        const size_t o = ((size_t)b * a.H + h) * a.Dv + 4 * tid;
+        const size_t o = ((size_t)b * a.H + h) * a.Dv + col;
         if (a.out_fp32) {
             *reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o) = sum;
         } else {
@@ -123,16 +127,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st)
 {
     const int R = a.mlra ? a.NU : 1;
-    const int V4 = a.Dv / 4;
-    const int G = kThreads / V4;
-    const size_t smem = (size_t)G * V4 * sizeof(float4) + (size_t)R * a.num_splits * sizeof(float);
+    const size_t smem = (size_t)R * a.num_splits * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess)
             return e;
     }
-    combine_kernel<<<dim3(a.H, a.B), kThreads, smem, st>>>(a);
+    combine_kernel<<<dim3(a.H, a.B, (a.Dv + kColsPerBlock - 1) / kColsPerBlock), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -41,21 +41,16 @@
 // drains its own copies and MMAs before it frees TMEM and exits.
 #include <math.h>
 
-#include "kvattn_internal.cuh"
-#include "sm100.cuh"
+#include "latent_common.cuh"
 
 namespace kvattn {
 
 namespace {
 
-constexpr int kRows = 128;                 // MMA M: query-head rows
+using namespace latent;
+
 constexpr int kSoftmaxThreads = 256;       // two warps per TMEM lane quarter
 constexpr int kThreads = 64 + kSoftmaxThreads;
-constexpr int kQChunkBytes = kRows * 128;  // 128 rows x 64 bf16, 128-byte swizzle
-constexpr float kLn2 = 0.69314718055994531f;
-constexpr float kRescaleThreshold = 8.f;   // log2 units
-
-constexpr int kMaxSplitPages = 1024;       // pages per part the page-validity table holds
 
 template <int T, int NKB, int STAGES, int NQT>
 struct LatentSmem {
@@ -76,34 +71,6 @@ struct LatentSmem {
     uint64_t xbar[4];                         // per lane quarter: the two threads of a row meet here
     uint32_t tmem_base;
 };
-
-__device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
-{
-    return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
-}
-
-__device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
-{
-    return page >= 0 && page < a.num_pages;
-}
-
-// Context tokens in tile j of the part starting at page p0 (0 if one of its
-// pages has a bad id); pvalid holds one bit per page of the part.
-template <int T>
-__device__ __forceinline__ int tile_ntok(const uint32_t *pvalid, int L, int p0, int j)
-{
-    constexpr int kSubs = T >= kPage ? T / kPage : 1;     // pages a tile spans
-    const int tok0 = p0 * kPage + j * T;
-    const int ntok = min(T, L - tok0);
-    bool ok = true;
-#pragma unroll
-    for (int sub = 0; sub < kSubs; ++sub) {
-        const int pg = (j * T) / kPage + sub;
-        if (sub * kPage < ntok)
-            ok = ok && ((pvalid[pg >> 5] >> (pg & 31)) & 1u);
-    }
-    return ok ? ntok : 0;
-}
 
 template <int T, int NKB, int NVB, int STAGES, int NQT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -565,10 +532,12 @@ int latent_tc_slots(const Problem &pr)
 cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_t st)
 {
     const int slots = latent_tc_slots(pr);
+    if (mla_pair_supported(pr))
+        return launch_mla_pair(a, st);
     if (pr.mlra)
         return launch_latent<128, 3, 2, 4, 3>(a, slots, st);
     if (pr.NU == 1)
-        return launch_latent<32, 9, 4, 4, 5>(a, slots, st);
+        return launch_latent<64, 9, 4, 2, 4>(a, slots, st);
     return launch_latent<64, 5, 4, 4, 4>(a, slots, st);
 }
 

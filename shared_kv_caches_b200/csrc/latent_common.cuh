@@ -1,0 +1,57 @@
+// Pieces shared by the tensor-core latent decode kernels (MLA, GLA, MLRA).
+#pragma once
+
+#include "kvattn_internal.cuh"
+#include "sm100.cuh"
+
+namespace kvattn {
+namespace latent {
+
+constexpr int kRows = 128;                 // MMA M: query-head rows
+constexpr int kQChunkBytes = kRows * 128;  // 128 rows x 64 bf16, 128-byte swizzle
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kRescaleThreshold = 8.f;   // log2 units: O is rescaled only past 2^8
+constexpr int kMaxSplitPages = 1024;       // pages per part the page-validity table holds
+
+__device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
+{
+    return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
+}
+
+__device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
+{
+    return page >= 0 && page < a.num_pages;
+}
+
+// Context tokens in tile j of the part starting at page p0 (0 if one of its
+// pages has a bad id); pvalid holds one bit per page of the part.
+template <int T>
+__device__ __forceinline__ int tile_ntok(const uint32_t *pvalid, int L, int p0, int j)
+{
+    constexpr int kSubs = T >= kPage ? T / kPage : 1;     // pages a tile spans
+    const int tok0 = p0 * kPage + j * T;
+    const int ntok = min(T, L - tok0);
+    bool ok = true;
+#pragma unroll
+    for (int sub = 0; sub < kSubs; ++sub) {
+        const int pg = (j * T) / kPage + sub;
+        if (sub * kPage < ntok)
+            ok = ok && ((pvalid[pg >> 5] >> (pg & 31)) & 1u);
+    }
+    return ok ? ntok : 0;
+}
+
+// Fill the page-validity bits of a part (threads [first, first + count)).
+__device__ __forceinline__ void fill_page_bits(uint32_t *pvalid, const DecodeArgs &a, int b, int p0, int npg,
+                                               int tid, int count)
+{
+    for (int w = tid; w < (npg + 31) / 32; w += count) {
+        uint32_t bits = 0;
+        for (int i = 32 * w; i < min(npg, 32 * w + 32); ++i)
+            bits |= (page_ok(a, page_id(a, b, p0 + i)) ? 1u : 0u) << (i & 31);
+        pvalid[w] = bits;
+    }
+}
+
+}  // namespace latent
+}  // namespace kvattn
