@@ -17,21 +17,32 @@ namespace kvattn {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kColsPerBlock = 32;          // value columns a block merges (8 float4)
-constexpr int kV4 = kColsPerBlock / 4;
-constexpr int kGroups = kThreads / kV4;    // row groups per block
+constexpr int kMaxV4 = kThreads;           // float4 columns a block can own
 
-// One block per (head, sequence, 32-column chunk of the value).  Warp 0 turns
-// the parts' lse values into merge weights (per branch for MLRA; every block
-// of a head recomputes them, which is cheap); then 16 groups of 8 threads
-// split the (branch, part) rows, each thread owning four value columns
-// (float4) with four row loads in flight; the groups meet in shared memory.
+// Row groups per block: enough to share the (branch, part) rows, at most 16,
+// a power of two; the block owns 4 * 128 / groups value columns.
+__host__ __device__ inline int combine_groups(int rows)
+{
+    int g = 1;
+    while (g < 16 && 2 * g <= rows)
+        g *= 2;
+    return g;
+}
+
+// One block per (head, sequence, chunk of value columns).  Warp 0 turns the
+// parts' lse values into merge weights (per branch for MLRA; every block of a
+// head recomputes them, which is cheap); then G groups of 128/G threads split
+// the (branch, part) rows, each thread owning four value columns (float4)
+// with four row loads in flight; the groups meet in shared memory.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
 {
     extern __shared__ float w_s[];     // [R][S] merge weights
-    __shared__ float4 acc_s[kGroups][kV4];
+    __shared__ float4 acc_s[kMaxV4];
     const int h = blockIdx.x, b = blockIdx.y;
-    const int c0 = blockIdx.z * kColsPerBlock;
+    const int R0 = a.mlra ? a.NU : 1;
+    const int kGroups = combine_groups(R0 * a.num_splits);
+    const int kV4 = kThreads / kGroups;
+    const int c0 = blockIdx.z * 4 * kV4;
     const int R = a.mlra ? a.NU : 1;
     const int S = a.num_splits;
     const int tid = threadIdx.x, lane = tid & 31;
@@ -97,12 +108,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
             acc.w = fmaf(w, v.w, acc.w);
         }
     }
-    acc_s[g][q4] = acc;
+    acc_s[g * kV4 + q4] = acc;
     __syncthreads();
     if (tid < kV4 && on) {
-        float4 sum = acc_s[0][tid];
+        float4 sum = acc_s[tid];
         for (int gg = 1; gg < kGroups; ++gg) {
-            const float4 v = acc_s[gg][tid];
+            const float4 v = acc_s[gg * kV4 + tid];
             sum.x += v.x;
             sum.y += v.y;
             sum.z += v.z;
@@ -134,7 +145,8 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st)
         if (e != cudaSuccess)
             return e;
     }
-    combine_kernel<<<dim3(a.H, a.B, (a.Dv + kColsPerBlock - 1) / kColsPerBlock), kThreads, smem, st>>>(a);
+    const int cols = 4 * (kThreads / combine_groups(R * a.num_splits));
+    combine_kernel<<<dim3(a.H, a.B, (a.Dv + cols - 1) / cols), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 

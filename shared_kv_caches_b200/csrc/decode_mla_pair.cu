@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_pair_kernel(const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.p_full[i], kSoftmaxThreads);
-            mbar_init(&S.xfull[i], kSoftmaxThreads);
+            mbar_init(&S.xfull[i], kSoftmaxThreads / 32);
         }
         mbar_init(&S.o_ready, 1);
         mbar_init(&S.q_ready, kSoftmaxThreads);
@@ -297,8 +297,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_pair_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < TH; i += 4)
                     st_cluster_f32x4(dst + 4 * i, s[i], s[i + 1], s[i + 2], s[i + 3]);
-                mbar_arrive_cluster(sb ? peer_xfull1 : peer_xfull0);
-                ok = __all_sync(0xffffffffu, mbar_wait_cluster(&S.xfull[sb], (j >> 1) & 1));
+                // one cluster-scope release per warp covers its lanes' stores (ordered
+                // by the warp barrier), and one lane polls the local barrier
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_cluster(sb ? peer_xfull1 : peer_xfull0);
+                bool got = true;
+                if (lane == 0)
+                    got = mbar_wait_cluster(&S.xfull[sb], (j >> 1) & 1);
+                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                __syncwarp();
                 if (!ok)
                     break;
                 const float4 *src = reinterpret_cast<const float4 *>(&S.recv[sb][h][half * TH]);
