@@ -19,14 +19,16 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kMaxV4 = kThreads;           // float4 columns a block can own
 
-// Row groups per block: enough to share the (branch, part) rows, at most 16,
-// a power of two; the block owns 4 * 128 / groups value columns.
-__host__ __device__ inline int combine_groups(int rows)
+// Row groups per block.  With many (branch, part) rows (long single
+// sequences) 16 groups share them and a block owns 32 value columns; with few
+// rows a block owns the whole value row (up to 512 columns) and the groups
+// split what is left of the 128 threads.
+__host__ __device__ inline int combine_groups(int rows, int dv)
 {
-    int g = 1;
-    while (g < 16 && 2 * g <= rows)
-        g *= 2;
-    return g;
+    if (rows >= 16)
+        return 16;
+    const int v4 = dv / 4;
+    return v4 >= kThreads ? 1 : kThreads / v4;
 }
 
 // One block per (head, sequence, chunk of value columns).  Warp 0 turns the
@@ -40,7 +42,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a)
     __shared__ float4 acc_s[kMaxV4];
     const int h = blockIdx.x, b = blockIdx.y;
     const int R0 = a.mlra ? a.NU : 1;
-    const int kGroups = combine_groups(R0 * a.num_splits);
+    const int kGroups = combine_groups(R0 * a.num_splits, a.Dv);
     const int kV4 = kThreads / kGroups;
     const int c0 = blockIdx.z * 4 * kV4;
     const int R = a.mlra ? a.NU : 1;
@@ -145,7 +147,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st)
         if (e != cudaSuccess)
             return e;
     }
-    const int cols = 4 * (kThreads / combine_groups(R * a.num_splits));
+    const int cols = 4 * (kThreads / combine_groups(R * a.num_splits, a.Dv));
     combine_kernel<<<dim3(a.H, a.B, (a.Dv + cols - 1) / cols), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

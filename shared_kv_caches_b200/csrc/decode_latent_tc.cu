@@ -532,8 +532,6 @@ int latent_tc_slots(const Problem &pr)
 cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_t st)
 {
     const int slots = latent_tc_slots(pr);
-    if (mla_pair_supported(pr))
-        return launch_mla_pair(a, st);
     if (pr.mlra)
         return launch_latent<128, 3, 2, 4, 3>(a, slots, st);
     if (pr.NU == 1)

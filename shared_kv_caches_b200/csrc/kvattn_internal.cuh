@@ -65,8 +65,6 @@ bool mqa_mma_supported(const Problem &pr);
 cudaError_t launch_mqa_mma(const DecodeArgs &a, cudaStream_t st);
 int latent_tc_slots(const Problem &pr);
 int latent_tc_page_multiple(const Problem &pr);
-bool mla_pair_supported(const Problem &pr);
-cudaError_t launch_mla_pair(const DecodeArgs &a, cudaStream_t st);
 int latent_tc_max_pages_per_split();
 cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_t st);
 
