@@ -19,13 +19,13 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kMaxV4 = kThreads;           // float4 columns a block can own
 
-// Row groups per block.  With many (branch, part) rows (long single
-// sequences) 16 groups share them and a block owns 32 value columns; with few
-// rows a block owns the whole value row (up to 512 columns) and the groups
-// split what is left of the 128 threads.
+// Row groups per block.  With many (branch, part) rows (a long single
+// sequence split over the whole GPU) 16 groups share them and a block owns 32
+// value columns; otherwise a block owns the whole value row (up to 512
+// columns) and the groups split what is left of the 128 threads.
 __host__ __device__ inline int combine_groups(int rows, int dv)
 {
-    if (rows >= 16)
+    if (rows >= 64)
         return 16;
     const int v4 = dv / 4;
     return v4 >= kThreads ? 1 : kThreads / v4;

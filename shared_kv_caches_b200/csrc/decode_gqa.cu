@@ -43,7 +43,7 @@ constexpr float kLn2 = 0.69314718055994531f;
 struct GqaSmem {
     unsigned char tiles[STAGES][STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
     float ow[CW][G][D];                         // per-warp outputs for the final merge
-    float2 pw[CW][TPW][G];                      // per-warp probabilities (each duplicated) of the page
+    float pw[CW][TPW][G];                       // per-warp probabilities of the current page
     float aw[CW][G];                            // per-warp rescale factors of the current page
     float mw[CW][G];
     float lw[CW][G];
@@ -55,22 +55,17 @@ struct GqaSmem {
 __device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// c += a * b on a pair of fp32 lanes (one packed FMA on sm_100).
-__device__ __forceinline__ void ffma2(float2 &c, float a0, float a1, float b0, float b1)
+__device__ __forceinline__ float dot8(const float *q, uint4 k)
 {
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-        : "+f"(c.x), "+f"(c.y)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
-// Pairwise partial dot of 8 query values with 8 bf16 keys into acc (two lanes).
-__device__ __forceinline__ void dot8x2(float2 &acc, const float *q, uint4 k)
-{
-    ffma2(acc, q[0], q[1], lo16(k.x), hi16(k.x));
-    ffma2(acc, q[2], q[3], lo16(k.y), hi16(k.y));
-    ffma2(acc, q[4], q[5], lo16(k.z), hi16(k.z));
-    ffma2(acc, q[6], q[7], lo16(k.w), hi16(k.w));
+    float s = q[0] * lo16(k.x);
+    s = fmaf(q[1], hi16(k.x), s);
+    s = fmaf(q[2], lo16(k.y), s);
+    s = fmaf(q[3], hi16(k.y), s);
+    s = fmaf(q[4], lo16(k.z), s);
+    s = fmaf(q[5], hi16(k.z), s);
+    s = fmaf(q[6], lo16(k.w), s);
+    s = fmaf(q[7], hi16(k.w), s);
+    return s;
 }
 
 __device__ __forceinline__ void load_q8(float *dst, const __nv_bfloat16 *src)
@@ -157,10 +152,10 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
         load_q8(q1[h], qr + 64 + 8 * j);
     }
     float m_run = -INFINITY, l_run = 0.f;
-    float2 O[G][2];
+    float O[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h)
-        O[h][0] = O[h][1] = make_float2(0.f, 0.f);
+        O[h][0] = O[h][1] = O[h][2] = O[h][3] = 0.f;
 
     const int t0 = warp * TPW;
     const int vbox = lane >> 4, vchunk = (lane & 15) >> 1, vhalf = lane & 1;
@@ -185,12 +180,8 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
                 const uint4 k1 = *reinterpret_cast<const uint4 *>(Kb + BOX_BYTES + off);
                 float part[G];
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float2 acc = make_float2(0.f, 0.f);
-                    dot8x2(acc, q0[h], k0);
-                    dot8x2(acc, q1[h], k1);
-                    part[h] = acc.x + acc.y;
-                }
+                for (int h = 0; h < G; ++h)
+                    part[h] = dot8(q0[h], k0) + dot8(q1[h], k1);
                 // transposing butterfly over the 8 lanes of this token
                 const bool up4 = (lane >> 2) & 1;
                 const float a0 = (up4 ? part[2] : part[0]) +
@@ -225,7 +216,7 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
             if ((lane & 1) == 0) {
 #pragma unroll
                 for (int it = 0; it < TPW / 4; ++it)
-                    S.pw[warp][4 * it + g][hh] = make_float2(sc[it], sc[it]);
+                    S.pw[warp][4 * it + g][hh] = sc[it];
                 if (lane < 8)
                     S.aw[warp][hh] = alpha;
             }
@@ -235,27 +226,22 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
             const float4 al = *reinterpret_cast<const float4 *>(S.aw[warp]);
             const float alv[G] = {al.x, al.y, al.z, al.w};
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                O[h][0].x *= alv[h];
-                O[h][0].y *= alv[h];
-                O[h][1].x *= alv[h];
-                O[h][1].y *= alv[h];
-            }
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    O[h][k] *= alv[h];
             const unsigned char *vrow = Vb + vbox * BOX_BYTES + vhalf * 8;
             for (int tl = 0; tl < nw; ++tl) {
                 const int t = t0 + tl;
                 const uint2 v = *reinterpret_cast<const uint2 *>(vrow + t * 128 + ((vchunk ^ (t & 7)) << 4));
-                const float4 p01 = *reinterpret_cast<const float4 *>(&S.pw[warp][tl][0]);
-                const float4 p23 = *reinterpret_cast<const float4 *>(&S.pw[warp][tl][2]);
-                const float v0 = lo16(v.x), v1 = hi16(v.x), v2 = lo16(v.y), v3 = hi16(v.y);
-                ffma2(O[0][0], p01.x, p01.y, v0, v1);
-                ffma2(O[0][1], p01.x, p01.y, v2, v3);
-                ffma2(O[1][0], p01.z, p01.w, v0, v1);
-                ffma2(O[1][1], p01.z, p01.w, v2, v3);
-                ffma2(O[2][0], p23.x, p23.y, v0, v1);
-                ffma2(O[2][1], p23.x, p23.y, v2, v3);
-                ffma2(O[3][0], p23.z, p23.w, v0, v1);
-                ffma2(O[3][1], p23.z, p23.w, v2, v3);
+                const float4 p4 = *reinterpret_cast<const float4 *>(S.pw[warp][tl]);
+                const float vv[4] = {lo16(v.x), hi16(v.x), lo16(v.y), hi16(v.y)};
+                const float pp[G] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        O[h][k] = fmaf(pp[h], vv[k], O[h][k]);
             }
         }
         __syncwarp();
@@ -270,7 +256,7 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
     }
 #pragma unroll
     for (int h = 0; h < G; ++h)
-        *reinterpret_cast<float4 *>(&S.ow[warp][h][4 * lane]) = make_float4(O[h][0].x, O[h][0].y, O[h][1].x, O[h][1].y);
+        *reinterpret_cast<float4 *>(&S.ow[warp][h][4 * lane]) = make_float4(O[h][0], O[h][1], O[h][2], O[h][3]);
     named_sync(1, CW * 32);
 
     const int tid = threadIdx.x;
