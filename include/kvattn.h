@@ -132,7 +132,8 @@ typedef struct {
     int32_t pages_per_split;   /* 64-token pages per part */
     int32_t ctas;              /* CTAs of the decode launch */
     int32_t launches;          /* kernel launches per kvattn_decode call */
-    int32_t reserved;
+    int32_t header_bytes;      /* leading workspace bytes that must be zero before a call
+                                  (error word and part counters); calls leave them zero */
     uint64_t workspace_bytes;  /* required workspace */
 } kvattn_plan;
 
@@ -141,22 +142,27 @@ typedef struct {
 int kvattn_get_plan(int32_t variant, const kvattn_params *p, kvattn_plan *plan);
 
 /* Bytes of workspace kvattn_decode needs for (variant, p): a 256-byte header
- * holding the device error word, then the per-part lse [B][splits][rows] and
- * normalised outputs [B][splits][rows][d_nope] in fp32 (rows = H, or H*R for
- * MLRA).  Host only. */
+ * holding the device error word, one counter per (sequence, KV head / unit)
+ * for kernels that merge their own parts, then the per-part lse
+ * [B][splits][rows] and normalised outputs [B][splits][rows][d_nope] in fp32
+ * (rows = H, or H*R for MLRA).  Host only. */
 int kvattn_workspace_size(int32_t variant, const kvattn_params *p, size_t *bytes);
 
-/* Zero the workspace header (device error word) on `stream`.  Call once
- * after allocating a workspace and after reading an error. */
+/* Zero the whole workspace on `stream`.  Call once after allocating a
+ * workspace, and again after a device error (a call cut short may leave its
+ * part counters non-zero). */
 int kvattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Decode attention, enqueued on `stream`: a split-KV pass that writes one
  * normalised partial output and lse per (sequence, head[, branch], part)
- * into the workspace, then a combine pass that merges the parts by their
- * lse (flash-decoding), sums the MLRA branches, places GLA group heads and
- * casts to out_dtype.  Returns KVATTN_OK once enqueued, a negative status
- * (nothing enqueued) for bad arguments, KVATTN_ERR_CUDA if a launch failed.
+ * into the workspace, and a merge of the parts by their lse
+ * (flash-decoding) that sums the MLRA branches, places GLA group heads and
+ * casts to out_dtype.  The GQA and MQA kernels merge in the last CTA of each
+ * (sequence, KV head) to finish (one launch); the others run a combine pass
+ * (two launches; kvattn_get_plan reports which).  Returns KVATTN_OK once
+ * enqueued, a negative status (nothing enqueued) for bad arguments,
+ * KVATTN_ERR_CUDA if a launch failed.
  */
 int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
                   const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
@@ -164,9 +170,10 @@ int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope, c
                   void *stream);
 
 /* kvattn_decode that also records caller-created cudaEvent_t handles on
- * `stream`: events[0] before the split pass, events[1] between the split pass
- * and the combine pass, events[2] after the combine pass (a NULL entry is
- * skipped; events may be NULL).  Used to time each pass on the launching
+ * `stream`: events[0] before the split pass, events[1] after it (for the
+ * kernels that merge their own parts this includes the merge), events[2]
+ * after the combine pass, or right after events[1] when there is none (a
+ * NULL entry is skipped; events may be NULL).  Used to time each pass on the launching
  * stream.  Same arguments, statuses and results as kvattn_decode. */
 int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_nope,
                         const void *q_rope, const void *kv_cache, const int32_t *block_table,

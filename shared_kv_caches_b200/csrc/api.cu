@@ -85,7 +85,9 @@ struct Plan {
     kvattn_plan pub;
     int head_chunk;
     int head_chunks;
+    size_t ticket_bytes;  // per (sequence, unit) part counters for in-kernel merges
     size_t lse_bytes;
+    bool fused_merge;     // the decode kernel merges its own parts (no combine launch)
 };
 
 // Parts per context: forced, or enough CTAs for several waves over the SMs
@@ -172,10 +174,13 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
     pl->pub.num_splits = splits;
     pl->pub.pages_per_split = pps;
     pl->pub.ctas = (int32_t)(base * splits);
-    pl->pub.launches = 2;
+    pl->fused_merge = pl->pub.kernel == KVATTN_KERNEL_GQA || pl->pub.kernel == KVATTN_KERNEL_MQA_TC;
+    pl->pub.launches = pl->fused_merge ? 1 : 2;
+    pl->ticket_bytes = align_up((size_t)pr.B * pr.NU * sizeof(int), 256);
+    pl->pub.header_bytes = (int32_t)(kWsHeader + pl->ticket_bytes);
     const size_t rows = (size_t)pr.B * splits * pr.HU;
     pl->lse_bytes = align_up(rows * sizeof(float), 256);
-    pl->pub.workspace_bytes = kWsHeader + pl->lse_bytes + rows * pr.Dv * sizeof(float);
+    pl->pub.workspace_bytes = kWsHeader + pl->ticket_bytes + pl->lse_bytes + rows * pr.Dv * sizeof(float);
     return KVATTN_OK;
 }
 
@@ -233,7 +238,7 @@ extern "C" int kvattn_workspace_init(void *workspace, size_t workspace_bytes, vo
         return KVATTN_ERR_INVALID_ARG;
     if (!aligned(workspace, 256))
         return KVATTN_ERR_MISALIGNED;
-    if (cudaMemsetAsync(workspace, 0, kWsHeader, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return KVATTN_ERR_CUDA;
     return KVATTN_OK;
 }
@@ -273,8 +278,12 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     a.block_table = block_table;
     a.seq_lens = seq_lens;
     a.err = reinterpret_cast<int *>(ws);
-    a.plse = reinterpret_cast<float *>(ws + kWsHeader);
-    a.po = reinterpret_cast<float *>(ws + kWsHeader + pl.lse_bytes);
+    a.tickets = reinterpret_cast<int *>(ws + kWsHeader);
+    a.plse = reinterpret_cast<float *>(ws + kWsHeader + pl.ticket_bytes);
+    a.po = reinterpret_cast<float *>(ws + kWsHeader + pl.ticket_bytes + pl.lse_bytes);
+    a.out = out;
+    a.lse_out = lse;
+    a.out_fp32 = pr.out_dtype == KVATTN_OUT_FP32;
     a.B = pr.B;
     a.H = pr.H;
     a.NU = pr.NU;
@@ -311,6 +320,8 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
         return KVATTN_ERR_CUDA;
     if (!mark(1))
         return KVATTN_ERR_CUDA;
+    if (pl.fused_merge)
+        return mark(2) ? KVATTN_OK : KVATTN_ERR_CUDA;
 
     CombineArgs c{};
     c.po = a.po;

@@ -50,6 +50,7 @@ struct GqaSmem {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     int skip[STAGES];
+    int last;
 };
 
 __device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
@@ -282,6 +283,11 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
             pl[h] = den > 0.f ? (mx + log2f(den)) * kLn2 : -INFINITY;
         }
     }
+
+    // the last part of (b, kvh) to finish merges all parts (the stage ring is
+    // free by now and serves as scratch for the merge weights)
+    if (finish_part(a, b * a.NU + kvh, &S.last, tid, CW * 32, 1))
+        merge_group(a, b, kvh * G, G, D, reinterpret_cast<float *>(S.tiles[0]), tid, CW * 32, 1);
 }
 
 }  // namespace
@@ -290,7 +296,9 @@ size_t gqa_smem_bytes() { return sizeof(GqaSmem) + 1024; }
 
 bool gqa_supported(const Problem &pr)
 {
-    return !pr.latent && pr.dn == D && pr.HPU == G && pr.mpps > 0;
+    // the in-kernel merge keeps G * splits weights in the stage ring
+    return !pr.latent && pr.dn == D && pr.HPU == G && pr.mpps > 0 &&
+           (size_t)G * kMaxSplits * sizeof(float) <= sizeof(GqaSmem::tiles);
 }
 
 cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st)

@@ -92,8 +92,9 @@ extern "C" int kvattn_decode_noalloc(int32_t variant, const kvattn_params *p, co
     if (st)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the device error word is the only part of the scratch that must start at zero
-    if (cudaMemsetAsync(scratch, 0, kWsHeader, s) != cudaSuccess)
+    // the device error word and the part counters are the only parts of the
+    // scratch that must start at zero
+    if (cudaMemsetAsync(scratch, 0, (size_t)plan.header_bytes, s) != cudaSuccess)
         return KVATTN_ERR_CUDA;
     st = kvattn_decode(variant, &q, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale, out,
                        lse, scratch, kNoallocScratchBytes, stream);

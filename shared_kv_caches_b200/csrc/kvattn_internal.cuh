@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include "kvattn.h"
@@ -38,6 +39,10 @@ struct DecodeArgs {
     float *po;
     float *plse;
     int *err;
+    int *tickets;                 // per (sequence, unit): parts finished (in-kernel merge)
+    void *out;                    // final output and lse, for kernels that merge their own parts
+    float *lse_out;
+    int out_fp32;
     int B, H, NU, dn, dr, row, HPU, HU;
     int mpps, num_pages, max_seq_len;
     int num_splits, pages_per_split, head_chunks;
@@ -54,6 +59,87 @@ struct CombineArgs {
 };
 
 __device__ __forceinline__ void raise_error(int *err, int bit) { atomicOr(err, bit); }
+
+// Merge of the parts of one (sequence b, rows hu0 .. hu0 + nrows - 1) group,
+// run by the last CTA of the group to finish: lse = ln sum_s exp(lse_s),
+// out = sum_s exp(lse_s - lse) o_s, cast to the output type.  w is shared
+// scratch of nrows * num_splits floats; tid / nthr index the threads taking
+// part, which meet at named barrier bar_id.  Partial rows written by other
+// CTAs are read past L1.
+__device__ __forceinline__ void merge_group(const DecodeArgs &a, int b, int hu0, int nrows, int Dv, float *w, int tid,
+                                            int nthr, int bar_id)
+{
+    const int S = a.num_splits;
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
+    for (int r = warp; r < nrows; r += nwarps) {
+        const float *pl = a.plse + (size_t)b * S * a.HU + hu0 + r;
+        float mx = -INFINITY;
+        for (int s = lane; s < S; s += 32)
+            mx = fmaxf(mx, __ldcg(pl + (size_t)s * a.HU));
+        for (int o = 16; o; o >>= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+        for (int s = lane; s < S; s += 32) {
+            const float e = mx == -INFINITY ? 0.f : expf(__ldcg(pl + (size_t)s * a.HU) - mx);
+            w[r * S + s] = e;
+            sum += e;
+        }
+        for (int o = 16; o; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = sum > 0.f ? 1.f / sum : 0.f;
+        for (int s = lane; s < S; s += 32)
+            w[r * S + s] *= inv;
+        if (lane == 0 && a.lse_out)
+            a.lse_out[(size_t)b * a.HU + hu0 + r] = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + logf(sum);
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthr) : "memory");
+    for (int idx = 4 * tid; idx < nrows * Dv; idx += 4 * nthr) {
+        const int r = idx / Dv, d = idx % Dv;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+            const float ws = w[r * S + s];
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                a.po + (((size_t)b * S + s) * a.HU + hu0 + r) * Dv + d));
+            acc.x = fmaf(ws, v.x, acc.x);
+            acc.y = fmaf(ws, v.y, acc.y);
+            acc.z = fmaf(ws, v.z, acc.z);
+            acc.w = fmaf(ws, v.w, acc.w);
+        }
+        const size_t o = ((size_t)b * a.H + hu0 + r) * Dv + d;
+        if (a.out_fp32) {
+            *reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o) = acc;
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 packed;
+            packed.x = *reinterpret_cast<const uint32_t *>(&lo);
+            packed.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.out) + o) = packed;
+        }
+    }
+}
+
+// Count this CTA's part of group `ticket_idx` as finished (after its partial
+// writes); true in the one CTA that finished last, which then owns the merge
+// and resets the counter for the next call.  All nthr threads call it.
+__device__ __forceinline__ bool finish_part(const DecodeArgs &a, int ticket_idx, int *flag, int tid, int nthr,
+                                            int bar_id)
+{
+    __threadfence();
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthr) : "memory");
+    if (tid == 0) {
+        const int t = atomicAdd(&a.tickets[ticket_idx], 1);
+        *flag = t == a.num_splits - 1;
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthr) : "memory");
+    const bool last = *flag != 0;
+    if (last) {
+        __threadfence();
+        if (tid == 0)
+            a.tickets[ticket_idx] = 0;
+    }
+    return last;
+}
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_generic(const DecodeArgs &a, int head_chunk, cudaStream_t st);

@@ -48,7 +48,7 @@ class kvattn_params(ctypes.Structure):
 class kvattn_plan(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("pages_per_split", ctypes.c_int32), ("ctas", ctypes.c_int32),
-                ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("header_bytes", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_uint64)]
 
 
