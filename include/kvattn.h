@@ -158,7 +158,7 @@ int kvattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
  * normalised partial output and lse per (sequence, head[, branch], part)
  * into the workspace, and a merge of the parts by their lse
  * (flash-decoding) that sums the MLRA branches, places GLA group heads and
- * casts to out_dtype.  The GQA and MQA kernels merge in the last CTA of each
+ * casts to out_dtype.  The GQA kernel merges in the last CTA of each
  * (sequence, KV head) to finish (one launch); the others run a combine pass
  * (two launches; kvattn_get_plan reports which).  Returns KVATTN_OK once
  * enqueued, a negative status (nothing enqueued) for bad arguments,

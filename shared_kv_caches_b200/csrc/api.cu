@@ -174,7 +174,9 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
     pl->pub.num_splits = splits;
     pl->pub.pages_per_split = pps;
     pl->pub.ctas = (int32_t)(base * splits);
-    pl->fused_merge = pl->pub.kernel == KVATTN_KERNEL_GQA || pl->pub.kernel == KVATTN_KERNEL_MQA_TC;
+    // the GQA kernel merges its own parts (a few KB per group); the MQA and
+    // latent groups are hundreds of KB to MB, merged faster by the combine grid
+    pl->fused_merge = pl->pub.kernel == KVATTN_KERNEL_GQA;
     pl->pub.launches = pl->fused_merge ? 1 : 2;
     pl->ticket_bytes = align_up((size_t)pr.B * pr.NU * sizeof(int), 256);
     pl->pub.header_bytes = (int32_t)(kWsHeader + pl->ticket_bytes);

@@ -43,7 +43,6 @@ struct MqaSmem {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     int skip[STAGES];
-    int last;
 };
 
 // Byte offset of 16-byte chunk c (8 dims) of token row t in a swizzled tile.
@@ -282,20 +281,13 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
         if (vh == 0 && c == 0)
             a.plse[rowbase + r + 8 * h] = l_run[h] > 0.f ? (m_run[h] + log2f(l_run[h])) * kLn2 : -INFINITY;
     }
-
-    // the last part of (b, kvh) to finish merges all parts (the stage ring is
-    // free by now and serves as scratch for the merge weights)
-    const int tid = threadIdx.x;
-    if (finish_part(a, b * a.NU + kvh, &S.last, tid, CW * 32, 1))
-        merge_group(a, b, kvh * HEADS, HEADS, D, reinterpret_cast<float *>(S.tiles[0]), tid, CW * 32, 1);
 }
 
 }  // namespace
 
 bool mqa_mma_supported(const Problem &pr)
 {
-    return !pr.latent && pr.dn == D && pr.HPU == HEADS &&
-           (size_t)HEADS * kMaxSplits * sizeof(float) <= sizeof(MqaSmem::tiles);
+    return !pr.latent && pr.dn == D && pr.HPU == HEADS;
 }
 
 cudaError_t launch_mqa_mma(const DecodeArgs &a, cudaStream_t st)
