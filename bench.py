@@ -95,15 +95,23 @@ def describe(names):
     return "; ".join(parts)
 
 
-def source_digest():
-    """sha256 over the CUDA sources, to tell whether a stored ncu traffic figure
-    still describes the kernels that run."""
+KERNEL_SOURCES = {
+    "gqa": ["decode_gqa.cu"],
+    "mqa_tc": ["decode_mqa_mma.cu"],
+    "latent_tc": ["decode_latent_tc.cu", "latent_common.cuh"],
+    "generic": ["decode_generic.cu"],
+}
+SHARED_SOURCES = ["kvattn_internal.cuh", "sm100.cuh"]
+
+
+def source_digest(kernel):
+    """sha256 prefix over a decode kernel's sources and the shared headers, to
+    tell whether a stored ncu traffic figure still describes that kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "shared_kv_caches_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -221,7 +229,7 @@ def run_ours(args, rank, world, local):
     t_s = decode_ms[dom] / 1e3
     t_mem = c["decode_bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = c["flops"] / (peaks["bf16_tflops"] * 1e12)
-    digest = source_digest()
+    digest = source_digest(probs[dom].plan_kernel_name())
     traffic = stored_traffic(args.workload, names[dom], digest)
     if t_tc > t_mem:
         achieved = c["flops"] / t_s / 1e12

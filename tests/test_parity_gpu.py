@@ -263,3 +263,34 @@ def test_sequence_longer_than_hint_sets_error_and_clamps(dev, oracle_mod):
     y = dict(x, seq_lens=np.array([200, 150], np.int32))
     ref_out, ref_lse = oracle_mod.decode(y)
     check(out, lse, ref_out, ref_lse, what="clamped")
+
+
+def test_timed_entry_point_records_ordered_events(dev):
+    """kvattn_decode_timed gives the same result as kvattn_decode and records
+    its three events in order on the launching stream."""
+    import torch
+    shape = SWEEP_SHAPES["mfa"].replace(batch=2, ctx=(300, 900))
+    x = W.make_inputs(shape, seed=10)
+    p, out_ref, lse_ref = run_gpu(x, dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for e in ev:
+        e.record()
+    p.out.zero_()
+    p.run(events=ev)
+    torch.cuda.synchronize()
+    out, lse = p.results()
+    np.testing.assert_array_equal(out, out_ref)
+    np.testing.assert_array_equal(lse, lse_ref)
+    assert ev[0].elapsed_time(ev[1]) > 0.0
+    assert ev[1].elapsed_time(ev[2]) >= 0.0
+
+
+def test_gqa_plan_merges_in_kernel(dev):
+    """The GQA kernel merges its own parts (one launch); the others use the combine pass."""
+    from shared_kv_caches_b200 import kvattn as K
+    for name, launches in (("gqa", 1), ("mfa", 2), ("mla", 2), ("mlra_128k", 2)):
+        s = W.WORKLOADS[name]
+        lo, hi = s.ctx
+        plan = K.kvattn_get_plan(s.variant_id, K.params_for(s, (hi + 63) // 64, 1 << 20, hi))
+        assert plan.launches == launches, name
+        assert plan.header_bytes >= 256
