@@ -9,16 +9,13 @@
 // Per CTA (part s of the context, KV head, sequence b): one producer warp
 // streams each 64-token page's K and V tiles (2 x 32 KB) into a STAGES-deep
 // ring with 3-D TMA loads (128-byte swizzle).  Four consumer warps split the
-// work as (16-head group) x (32-token half of the page): each forms the
-// 16 x 32 score tile of its heads and tokens once, keeps its own
-// online-softmax state for its 16 rows (fp32, base 2), turns the scores into
-// the bf16 A operand of P.V in registers and accumulates a full 16 x 256
-// output.  The query tile lives in shared memory (read with ldmatrix), which
-// leaves room in the registers for that output.  At the end of the part the
-// two token halves of each head group are merged by their max, the same LSE
-// merge the combine pass applies across parts.  Token slots past the context
-// are masked in the scores and their value rows are zeroed in shared memory,
-// since 0 * NaN would still poison an MMA.
+// work as (16-head group) x (128-dim half of the value): each computes the
+// 16 x 64 score tile of its heads (the two warps of a head group both do, so
+// no scores cross warps), keeps the online-softmax state of its 16 rows in
+// registers (fp32, base 2), turns the scores into the bf16 A operand of P.V
+// in registers, and accumulates its 16 x 128 output slice.  Token slots past
+// the context are masked in the scores and their value rows are zeroed in
+// shared memory first, since 0 * NaN would still poison an MMA.
 #include <math.h>
 
 #include "kvattn_internal.cuh"
@@ -31,23 +28,18 @@ namespace {
 constexpr int D = 256;
 constexpr int HEADS = 32;
 constexpr int HG = HEADS / 16;               // 16-head groups
-constexpr int TH = 2;                        // token halves of a page
-constexpr int TPH = kPage / TH;              // tokens per half
-constexpr int CW = HG * TH;                  // consumer warps
+constexpr int VH = D / 128;                  // 128-dim value slices
+constexpr int CW = HG * VH;                  // consumer warps
 constexpr int THREADS = (CW + 1) * 32;
 constexpr int STAGES = 3;
 constexpr int BOX_BYTES = kPage * 64 * 2;    // 64 tokens x 64 dims
 constexpr int TILE_BYTES = (D / 64) * BOX_BYTES;
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;
 constexpr int KSTEPS = D / 16;
-constexpr int NT_O = D / 8;                  // output n-tiles (8 dims each)
 constexpr float kLn2 = 0.69314718055994531f;
 
 struct MqaSmem {
     unsigned char tiles[STAGES][STAGE_BYTES];
-    unsigned char q[HEADS * D * 2];            // [head][dim] bf16, 16-byte chunks XOR-swizzled by row
-    float mstate[HG][TH][16];                  // end-of-part merge: per-row max and sum
-    float lstate[HG][TH][16];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     int skip[STAGES];
@@ -57,12 +49,6 @@ struct MqaSmem {
 __device__ __forceinline__ uint32_t chunk_off(int t, int c)
 {
     return (uint32_t)((c >> 3) * BOX_BYTES + t * 128 + (((c & 7) ^ (t & 7)) << 4));
-}
-
-// Byte offset of 16-byte chunk c of query row h (rows are 512 bytes).
-__device__ __forceinline__ uint32_t q_off(int h, int c)
-{
-    return (uint32_t)(h * (D * 2) + (((c & ~7) | ((c & 7) ^ (h & 7))) << 4));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
@@ -154,30 +140,30 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
         return;
     }
 
-    const int tid = threadIdx.x;
-    const int hg = warp % HG, th = warp / HG;
+    const int hg = warp % HG, vh = warp / HG;
     const int r = lane >> 2, c = lane & 3;
-    const int mrow = lane & 7, mat = lane >> 3;
+    const int head0 = kvh * HEADS + hg * 16;
 
-    // the query tile of this KV head's 32 heads into shared memory
+    // Q fragments of this warp's 16 heads over the whole head dim (A operand)
+    uint32_t qf[KSTEPS][4];
     {
-        const __nv_bfloat16 *qsrc = a.q_nope + ((size_t)b * a.H + (size_t)kvh * HEADS) * D;
-        for (int idx = tid; idx < HEADS * D / 8; idx += CW * 32) {
-            const int h = idx / (D / 8), cc = idx % (D / 8);
-            *reinterpret_cast<uint4 *>(S.q + q_off(h, cc)) =
-                *reinterpret_cast<const uint4 *>(qsrc + (size_t)h * D + 8 * cc);
-        }
-        named_sync(1, CW * 32);
-    }
-    const uint32_t qbase = smem_u32(S.q);
-
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-    float o[NT_O][4];
+        const __nv_bfloat16 *q0 = a.q_nope + ((size_t)b * a.H + head0 + r) * D;
+        const __nv_bfloat16 *q8 = q0 + 8 * D;
 #pragma unroll
-    for (int nt = 0; nt < NT_O; ++nt)
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + 16 * kk + 2 * c);
+            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + 16 * kk + 2 * c);
+            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + 16 * kk + 8 + 2 * c);
+            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + 16 * kk + 8 + 2 * c);
+        }
+    }
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
         o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
 
-    const int t0 = th * TPH;
+    const int mrow = lane & 7, mat = lane >> 3;
     for (int i = 0; i < n; ++i) {
         const int st = i % STAGES;
         if (!mbar_wait(&S.full[st], (i / STAGES) & 1)) {
@@ -186,47 +172,44 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
             break;
         }
         const int ntok = S.skip[st] ? 0 : min(kPage, L - (p0 + i) * kPage);
-        const int nh = min(max(ntok - t0, 0), TPH);          // context tokens in this warp's half
         unsigned char *Kb = S.tiles[st];
         unsigned char *Vb = Kb + TILE_BYTES;
-        if (nh > 0 && nh < TPH) {
-            // zero the value rows of this half past the context (the two head
-            // groups of the half write the same zeros, then both wait)
-            for (int idx = lane + 32 * hg; idx < (TPH - nh) * (D / 8); idx += 32 * HG) {
-                const int t = t0 + nh + idx / (D / 8), cc = idx % (D / 8);
+        if (ntok > 0 && ntok < kPage) {
+            // zero this warp's value slice of the slots past the context (the two
+            // warps of a value half write the same zeros, then both wait)
+            for (int idx = lane + 32 * hg; idx < (kPage - ntok) * 16; idx += 32 * HG) {
+                const int t = ntok + idx / 16, cc = vh * 16 + (idx % 16);
                 *reinterpret_cast<uint4 *>(Vb + chunk_off(t, cc)) = make_uint4(0, 0, 0, 0);
             }
-            named_sync(2 + th, 32 * HG);
+            named_sync(2 + vh, 32 * HG);
         }
-        if (nh > 0) {
+        if (ntok > 0) {
             const uint32_t kbase = smem_u32(Kb), vbase = smem_u32(Vb);
-            // S = Q K^T for 16 heads x 32 tokens
-            float s[4][4];
+            // S = Q K^T for 16 heads x 64 tokens
+            float s[8][4];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 8; ++nt)
                 s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
-                uint32_t qa[4];
-                ldsm_x4(qbase + q_off(hg * 16 + (mat & 1) * 8 + mrow, 2 * kk + (mat >> 1)), qa[0], qa[1], qa[2],
-                        qa[3]);
 #pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    const int t = t0 + np * 16 + (mat >> 1) * 8 + mrow;
+                for (int np = 0; np < 4; ++np) {
+                    const int t = np * 16 + (mat >> 1) * 8 + mrow;
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4(kbase + chunk_off(t, 2 * kk + (mat & 1)), b0, b1, b2, b3);
-                    mma_bf16(s[2 * np], qa, b0, b1);
-                    mma_bf16(s[2 * np + 1], qa, b2, b3);
+                    mma_bf16(s[2 * np], qf[kk], b0, b1);
+                    mma_bf16(s[2 * np + 1], qf[kk], b2, b3);
                 }
             }
-            // online softmax on rows r and r + 8 of this warp's tokens
+            // online softmax on rows r and r + 8
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int nt = 0; nt < 8; ++nt) {
+                const int t = nt * 8 + 2 * c;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int tt = nt * 8 + 2 * c + (e & 1);
-                    s[nt][e] = tt < nh ? s[nt][e] * a.scale_log2 : -INFINITY;
+                    const int tt = t + (e & 1);
+                    s[nt][e] = tt < ntok ? s[nt][e] * a.scale_log2 : -INFINITY;
                     mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
                 }
             }
@@ -241,9 +224,9 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
                 m_run[h] = m_new;
             }
             float ps[2] = {0.f, 0.f};
-            uint32_t pf[2][4];
+            uint32_t pf[4][4];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     s[nt][e] = exp2f(s[nt][e] - m_use[e >> 1]);
@@ -260,19 +243,19 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
                 l_run[h] = l_run[h] * alpha[h] + ps[h];
             }
 #pragma unroll
-            for (int nt = 0; nt < NT_O; ++nt) {
+            for (int nt = 0; nt < 16; ++nt) {
                 o[nt][0] *= alpha[0];
                 o[nt][1] *= alpha[0];
                 o[nt][2] *= alpha[1];
                 o[nt][3] *= alpha[1];
             }
-            // O += P V over all 256 value dims and this warp's 32 tokens
+            // O += P V over this warp's 128 value dims
 #pragma unroll
-            for (int kk = 0; kk < TPH / 16; ++kk) {
-                const int t = t0 + kk * 16 + (mat & 1) * 8 + mrow;
+            for (int kk = 0; kk < 4; ++kk) {
+                const int t = kk * 16 + (mat & 1) * 8 + mrow;
 #pragma unroll
-                for (int np = 0; np < NT_O / 2; ++np) {
-                    const int cc = np * 2 + (mat >> 1);
+                for (int np = 0; np < 8; ++np) {
+                    const int cc = vh * 16 + np * 2 + (mat >> 1);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_t(vbase + chunk_off(t, cc), b0, b1, b2, b3);
                     mma_bf16(o[2 * np], pf[kk], b0, b1);
@@ -285,45 +268,18 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
             mbar_arrive(&S.empty[st]);
     }
 
-    // merge the two token halves of each head group: the th = 1 warp hands its
-    // state over through shared memory (the stage ring is free by now)
-    named_sync(1, CW * 32);
-    float *ox = reinterpret_cast<float *>(S.tiles[0]) + (size_t)hg * 16 * D;   // [16][256] per head group
-    if (th == 1) {
+    // this warp's 16 heads x 128 dims of the part result
+    const size_t rowbase = ((size_t)b * a.num_splits + split) * a.HU + head0;
 #pragma unroll
-        for (int nt = 0; nt < NT_O; ++nt) {
-            *reinterpret_cast<float2 *>(ox + (size_t)r * D + nt * 8 + 2 * c) = make_float2(o[nt][0], o[nt][1]);
-            *reinterpret_cast<float2 *>(ox + (size_t)(r + 8) * D + nt * 8 + 2 * c) = make_float2(o[nt][2], o[nt][3]);
-        }
-        if (c == 0) {
-            S.mstate[hg][1][r] = m_run[0];
-            S.mstate[hg][1][r + 8] = m_run[1];
-            S.lstate[hg][1][r] = l_run[0];
-            S.lstate[hg][1][r + 8] = l_run[1];
-        }
-    }
-    named_sync(1, CW * 32);
-    if (th == 0) {
-        const size_t rowbase = ((size_t)b * a.num_splits + split) * a.HU + (size_t)kvh * HEADS + hg * 16;
+    for (int h = 0; h < 2; ++h) {
+        const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+        float *dst = a.po + (rowbase + r + 8 * h) * D + vh * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int row = r + 8 * h;
-            const float m1 = S.mstate[hg][1][row], l1 = S.lstate[hg][1][row];
-            const float mm = fmaxf(m_run[h], m1);
-            const float w0 = mm == -INFINITY ? 0.f : exp2f(m_run[h] - mm);
-            const float w1 = mm == -INFINITY ? 0.f : exp2f(m1 - mm);
-            const float l = w0 * l_run[h] + w1 * l1;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            float *dst = a.po + (rowbase + row) * D;
-#pragma unroll
-            for (int nt = 0; nt < NT_O; ++nt) {
-                const float2 x = *reinterpret_cast<const float2 *>(ox + (size_t)row * D + nt * 8 + 2 * c);
-                *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
-                    make_float2((w0 * o[nt][2 * h] + w1 * x.x) * inv, (w0 * o[nt][2 * h + 1] + w1 * x.y) * inv);
-            }
-            if (c == 0)
-                a.plse[rowbase + row] = l > 0.f ? (mm + log2f(l)) * kLn2 : -INFINITY;
-        }
+        for (int nt = 0; nt < 16; ++nt)
+            *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
+                make_float2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
+        if (vh == 0 && c == 0)
+            a.plse[rowbase + r + 8 * h] = l_run[h] > 0.f ? (m_run[h] + log2f(l_run[h])) * kLn2 : -INFINITY;
     }
 }
 
