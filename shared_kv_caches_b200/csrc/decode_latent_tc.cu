@@ -21,14 +21,23 @@
 // columns: two score / probability buffers of T, the output slice, the Q
 // chunks (MLRA 256 + 128 + 96, MLA and GLA 128 + 256 + 128).
 //
-// Warp roles (192 threads):
-//   warp 0     TMEM allocation; one thread streams each tile's key boxes into
-//              a STAGES-deep shared-memory ring with 2-D TMA loads (128-byte
-//              swizzle, completion on kv_full; a 128-token tile is two pages)
-//   warp 1     one thread issues S_j = Q K_j^T into one of two TMEM score
-//              buffers, then P_{j-1} V_{j-1} into the TMEM output; the warp
-//              zeroes the rows of a tile past the context first (0 * NaN
-//              would poison the MMA)
+// A stage of the shared-memory ring holds one tile's key boxes in two
+// groups with their own barriers: the E boxes (key columns that are not this
+// slot's values: the rope key, and for MLA the other value half) are free
+// again as soon as the score MMAs that read them complete, the V boxes (this
+// slot's value columns) only after P.V.  The next tiles' E boxes therefore
+// load while a tile's softmax and P.V run, and a V group has the MMAs of a
+// whole tile to land in.
+//
+// Warp roles (320 threads):
+//   warp 0     TMEM allocation; one thread streams each tile's E group, then
+//              its V group, into a STAGES-deep ring with 2-D TMA loads
+//              (128-byte swizzle; a 128-token tile is two pages)
+//   warp 1     one thread issues the E part of S_j = Q K_j^T into one of two
+//              TMEM score buffers, then, in whichever order their inputs
+//              arrive, the V part of S_j and P_{j-1} V_{j-1} into the TMEM
+//              output; the warp zeroes the rows of a tile past the context
+//              first (0 * NaN would poison the MMA)
 //   warps 2-9  two threads per head row, each owning half of the tile's
 //              columns and half of O's: read S_j from TMEM, exchange the tile
 //              maximum with the partner thread through shared memory, online
@@ -40,6 +49,8 @@
 // Every wait is bounded; a wait that gives up sets an error bit and the CTA
 // drains its own copies and MMAs before it frees TMEM and exits.
 #include <math.h>
+
+#include <type_traits>
 
 #include "latent_common.cuh"
 
@@ -61,8 +72,10 @@ struct LatentSmem {
     unsigned char kv[STAGES][kStageBytes];
     float xmax[2][2][kRows];                  // [exchange parity][column half][row]
     uint32_t pvalid[kMaxSplitPages / 32];     // one bit per page of the part
-    uint64_t kv_full[STAGES];
-    uint64_t kv_empty[STAGES];
+    uint64_t e_full[STAGES];                  // E group of the stage landed
+    uint64_t v_full[STAGES];                  // V group landed
+    uint64_t e_empty[STAGES];                 // score MMAs done with the E group
+    uint64_t v_empty[STAGES];                 // P.V done with the V group
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_ready;
@@ -97,6 +110,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     const int dn_boxes = a.dn / 64;
+    constexpr int NE = NKB - NVB;                                // E boxes: stage positions 0..NE-1
+    // Split release pays when the ring is shallow (MLA: two stages of nine
+    // boxes); with a deep ring and a one-box E group the whole stage is one
+    // group: loaded on e_full, freed by P.V on e_empty.
+    constexpr bool kSplit = NE > 1;
+    // Key box (64-column block of the slot's key row) at stage position p:
+    // E positions first (MLA: the other value half, then the rope key;
+    // GLA and MLRA: the rope key), the slot's value columns last.
+    auto key_box = [&](int p) -> int {
+        if (mla)
+            return p < NVB ? (slot ^ 1) * NVB + p : (p == NVB ? 2 * NVB : slot * NVB + (p - NE));
+        return p < NE ? NVB + p : p - NE;
+    };
 
     int L = a.seq_lens[b];
     if (L > a.max_seq_len) {
@@ -111,8 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
-            mbar_init(&S.kv_full[st], 1);
-            mbar_init(&S.kv_empty[st], 1);
+            mbar_init(&S.e_full[st], 1);
+            mbar_init(&S.v_full[st], 1);
+            mbar_init(&S.e_empty[st], 1);
+            mbar_init(&S.v_empty[st], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
@@ -140,16 +168,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && n > 0) {
             prefetch_tmap(&kv_map);
             const int unit_col0 = mla ? 0 : slot * a.dn;
-            int issued = 0;
-            for (int j = 0; j < n; ++j) {
-                const int st = j % STAGES;
-                if (j >= STAGES && !mbar_wait(&S.kv_empty[st], ((j / STAGES) - 1) & 1)) {
-                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                    break;
-                }
-                issued = j + 1;
-                constexpr int kSubs = T >= kPage ? T / kPage : 1;   // pages a tile spans
-                constexpr int kSubRows = T >= kPage ? kPage : T;    // rows per TMA box
+            constexpr int kSubs = T >= kPage ? T / kPage : 1;   // pages a tile spans
+            constexpr int kSubRows = T >= kPage ? kPage : T;    // rows per TMA box
+            int e_issued = 0, v_issued = 0;                     // tiles whose E / V group was started
+            // Start one group (positions [p_lo, p_hi)) of tile j on stage st;
+            // a tile with a bad page id loads nothing and only arrives.
+            auto load_group = [&](int j, int st, int p_lo, int p_hi, uint64_t *full) {
                 const int tok0 = p0 * kPage + j * T;
                 const int ntok = min(T, L - tok0);
                 const int nsub = (ntok + kSubRows - 1) / kSubRows;  // boxes of this tile holding context
@@ -162,101 +186,228 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                 }
                 if (!ok) {
-                    if (slot == 0)
+                    if (slot == 0 && p_lo == 0)
                         raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);
-                    mbar_arrive(&S.kv_full[st]);
-                    continue;
+                    mbar_arrive(full);
+                    return;
                 }
-                mbar_arrive_expect_tx(&S.kv_full[st], (uint32_t)(nsub * NKB * kSubRows * 128));
+                mbar_arrive_expect_tx(full, (uint32_t)(nsub * (p_hi - p_lo) * kSubRows * 128));
                 const int off = tok0 % kPage;
 #pragma unroll
                 for (int sub = 0; sub < kSubs; ++sub) {
                     if (sub >= nsub)
                         break;
                     const int y = (int)(pages[sub] * kPage) + off;
-#pragma unroll
-                    for (int i = 0; i < NKB; ++i) {
-                        const int col = i < dn_boxes ? unit_col0 + 64 * i : a.NU * a.dn + 64 * (i - dn_boxes);
-                        tma_load_2d(S.kv[st] + i * kBoxBytes + sub * kSubRows * 128, &kv_map, col, y, &S.kv_full[st]);
+                    for (int p = p_lo; p < p_hi; ++p) {
+                        const int kb = key_box(p);
+                        const int col = kb < dn_boxes ? unit_col0 + 64 * kb : a.NU * a.dn + 64 * (kb - dn_boxes);
+                        tma_load_2d(S.kv[st] + p * kBoxBytes + sub * kSubRows * 128, &kv_map, col, y, full);
+                    }
+                }
+            };
+            if constexpr (!kSplit) {
+                for (; e_issued < n; ++e_issued) {
+                    const int j = e_issued, st = j % STAGES;
+                    if (j >= STAGES && !mbar_wait(&S.e_empty[st], ((j / STAGES) - 1) & 1)) {
+                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                        break;
+                    }
+                    load_group(j, st, 0, NKB, &S.e_full[st]);
+                }
+                v_issued = 0;
+            } else {
+                // E groups may run ahead of V groups: each group waits only for
+                // its own slot; the lower tile goes first when both can
+                uint32_t idle = 0;
+                while (v_issued < n) {
+                    const bool v_can = v_issued < e_issued &&
+                                       (v_issued < STAGES ||
+                                        mbar_test(&S.v_empty[v_issued % STAGES], ((v_issued / STAGES) - 1) & 1));
+                    if (v_can) {
+                        load_group(v_issued, v_issued % STAGES, NE, NKB, &S.v_full[v_issued % STAGES]);
+                        ++v_issued;
+                        idle = 0;
+                        continue;
+                    }
+                    const bool e_can = e_issued < n &&
+                                       (e_issued < STAGES ||
+                                        mbar_test(&S.e_empty[e_issued % STAGES], ((e_issued / STAGES) - 1) & 1));
+                    if (e_can) {
+                        load_group(e_issued, e_issued % STAGES, 0, NE, &S.e_full[e_issued % STAGES]);
+                        ++e_issued;
+                        idle = 0;
+                        continue;
+                    }
+                    if (++idle >= kWaitLimit) {
+                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                        break;
                     }
                 }
             }
             // every copy this thread started has landed before the CTA can exit
-            for (int st = 0; st < STAGES && st < issued; ++st) {
-                const int jl = st + ((issued - 1 - st) / STAGES) * STAGES;
-                if (!mbar_wait(&S.kv_full[st], (jl / STAGES) & 1))
-                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+            for (int st = 0; st < STAGES; ++st) {
+                if (st < e_issued) {
+                    const int jl = st + ((e_issued - 1 - st) / STAGES) * STAGES;
+                    if (!mbar_wait(&S.e_full[st], (jl / STAGES) & 1))
+                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                }
+                if (st < v_issued) {
+                    const int jl = st + ((v_issued - 1 - st) / STAGES) * STAGES;
+                    if (!mbar_wait(&S.v_full[st], (jl / STAGES) & 1))
+                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         const uint32_t qbase = smem_u32(&S.q[0][0]);
-        bool ok = mbar_wait(&S.q_ready, 0);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&S.q_ready, 0));
         tc_fence_after();
-        auto issue_pv = [&](int t) -> bool {
-            if (!mbar_wait(&S.p_full[t & 1], (t >> 1) & 1))
-                return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t vbase = smem_u32(S.kv[t % STAGES]) + (mla ? slot * NVB : 0) * kBoxBytes;
-#pragma unroll
-                for (int k = 0; k < T / 16; ++k) {
-                    const uint64_t vd = smem_desc(vbase + k * 16 * 128, kBoxBytes, 1024, 2);
-                    umma_ts(tO, tS + (t & 1) * T + 8 * k, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
-                }
-                umma_commit(&S.o_ready);
-                umma_commit(&S.kv_empty[t % STAGES]);
-            }
-            __syncwarp();
-            return true;
+        // lane 0 (the issuing thread) tests a barrier; the warp follows its view
+        auto test = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __shfl_sync(0xffffffffu, (lane == 0 && mbar_test(bar, parity)) ? 1 : 0, 0) != 0;
         };
-        int j = 0;
-        for (; ok && j < n; ++j) {
-            const int st = j % STAGES;
-            if (!mbar_wait(&S.kv_full[st], (j / STAGES) & 1)) {
-                ok = false;
-                break;
+        // zero rows [ntok, T) of stage positions [p_lo, p_hi) once the group's
+        // copies (whole boxes, rows past the context included) have landed;
+        // every lane observes the completed phase before it writes
+        auto zero_tail = [&](int st, int ntok, int p_lo, int p_hi, uint64_t *full, uint32_t parity) {
+            if (ntok >= T)
+                return;
+            mbar_wait(full, parity);
+            const int rows = T - ntok, nb = p_hi - p_lo;
+            for (int idx = lane; idx < rows * nb * 8; idx += 32) {
+                const int box = p_lo + idx / (rows * 8), rem = idx % (rows * 8);
+                const int row = ntok + rem / 8, piece = rem % 8;
+                *reinterpret_cast<uint4 *>(S.kv[st] + box * kBoxBytes + row * 128 + piece * 16) =
+                    make_uint4(0, 0, 0, 0);
             }
-            const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
-            if (ntok < T) {
-                // zero the rows past the context in every key box of the stage
-                const int rows = T - ntok;
-                for (int idx = lane; idx < rows * NKB * 8; idx += 32) {
-                    const int box = idx / (rows * 8), rem = idx % (rows * 8);
-                    const int row = ntok + rem / 8, piece = rem % 8;
-                    *reinterpret_cast<uint4 *>(S.kv[st] + box * kBoxBytes + row * 128 + piece * 16) =
-                        make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            tc_fence_after();
+            fence_proxy_async_smem();
+            __syncwarp();
+        };
+        // Descriptors are built once; a byte offset moves the start-address
+        // field by offset >> 4 (shared addresses stay below 256 KB, so the
+        // 14-bit field never carries).  The issuing thread does a few integer
+        // adds per MMA: with narrow score tiles the MMAs are short and the
+        // single issuing thread would otherwise set the pace.
+        constexpr uint32_t kStageUnits = Smem::kStageBytes >> 4, kBoxUnits = kBoxBytes >> 4;
+        const uint64_t kdesc0 = smem_desc(smem_u32(S.kv[0]), 16, 1024, 2);                      // K-major key boxes
+        const uint64_t vdesc0 = smem_desc(smem_u32(S.kv[0]) + NE * kBoxBytes, kBoxBytes, 1024, 2);  // MN-major values
+        const uint64_t qdesc0 = smem_desc(qbase, 16, 1024, 2);
+        // score MMAs of stage positions [PLO, PHI) of tile j
+        auto issue_s = [&](int j, auto PLO, auto PHI) {
             if (lane == 0) {
-                const uint32_t kbase = smem_u32(S.kv[st]);
+                const uint32_t d = tS + (j & 1) * T;
+                const uint64_t kd = kdesc0 + (uint64_t)((j % STAGES) * kStageUnits);
 #pragma unroll
-                for (int kb = 0; kb < NKB; ++kb) {
+                for (int p = decltype(PLO)::value; p < decltype(PHI)::value; ++p) {
+                    const int kb = key_box(p);
+                    if (kb < NQT) {
+                        const uint32_t qa = tQ + kb * 32;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t kd = smem_desc(kbase + kb * kBoxBytes + k * 32, 16, 1024, 2);
-                        if (kb < NQT) {
-                            umma_ts(tS + (j & 1) * T, tQ + kb * 32 + k * 8, kd, kIdescS, (kb | k) ? 1u : 0u);
-                        } else {
-                            const uint64_t qd = smem_desc(qbase + (kb - NQT) * kQChunkBytes + k * 32, 16, 1024, 2);
-                            umma_ss(tS + (j & 1) * T, qd, kd, kIdescS, (kb | k) ? 1u : 0u);
-                        }
+                        for (int k = 0; k < 4; ++k)
+                            umma_ts(d, qa + k * 8, kd + (uint64_t)(p * kBoxUnits + k * 2), kIdescS, (p | k) ? 1u : 0u);
+                    } else {
+                        const uint64_t qd = qdesc0 + (uint64_t)((kb - NQT) * (kQChunkBytes >> 4));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            umma_ss(d, qd + (uint64_t)(k * 2), kd + (uint64_t)(p * kBoxUnits + k * 2), kIdescS,
+                                    (p | k) ? 1u : 0u);
                     }
                 }
-                umma_commit(&S.s_full[j & 1]);
+            }
+        };
+        using P0 = std::integral_constant<int, 0>;
+        using PE = std::integral_constant<int, NE>;
+        using PK = std::integral_constant<int, NKB>;
+        // P_t V_t into O (P_t is ready); frees tile t's V group
+        auto issue_pv = [&](int t) {
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t vd = vdesc0 + (uint64_t)((t % STAGES) * kStageUnits);
+                const uint32_t pa = tS + (t & 1) * T;
+#pragma unroll
+                for (int k = 0; k < T / 16; ++k)
+                    umma_ts(tO, pa + 8 * k, vd + (uint64_t)(k * 128), kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&S.o_ready);
+                umma_commit(kSplit ? &S.v_empty[t % STAGES] : &S.e_empty[t % STAGES]);
             }
             __syncwarp();
-            if (j >= 1 && !issue_pv(j - 1)) {
-                ok = false;
-                break;
+        };
+        if constexpr (!kSplit) {
+            // S_j as soon as its stage is in, then P_{j-1} V_{j-1}
+            for (int j = 0; ok && j < n; ++j) {
+                const int st = j % STAGES;
+                const uint32_t fph = (j / STAGES) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&S.e_full[st], fph))) {
+                    ok = false;
+                    break;
+                }
+                zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, j), 0, NKB, &S.e_full[st], fph);
+                tc_fence_after();
+                issue_s(j, P0{}, PK{});
+                if (lane == 0)
+                    umma_commit(&S.s_full[j & 1]);
+                __syncwarp();
+                if (j >= 1) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&S.p_full[(j - 1) & 1], ((j - 1) >> 1) & 1)))
+                        ok = false;
+                    else
+                        issue_pv(j - 1);
+                }
+            }
+            if (ok && n > 0) {
+                if (__all_sync(0xffffffffu, mbar_wait(&S.p_full[(n - 1) & 1], ((n - 1) >> 1) & 1)))
+                    issue_pv(n - 1);
+                else
+                    ok = false;
+            }
+        } else {
+            // Three kinds of work, issued as their inputs arrive (the V part of
+            // the open score tile first, so its softmax starts early, then P.V,
+            // then the next tile's E part):
+            //   PV_t     needs P_t (so S_t is complete)
+            //   S_t(V)   needs the V group of tile t and S_t(E)
+            //   S_t(E)   needs the E group of tile t, S_{t-1}(V) (scores complete in
+            //            tile order) and PV_{t-2} (S_t reuses the buffer P_{t-2} was in;
+            //            MMAs run in issue order)
+            int jpv = 0, jsv = 0, jse = 0;             // next tile of each kind
+            uint32_t idle = 0;
+            while (ok && jpv < n) {
+                if (jsv < jse && test(&S.v_full[jsv % STAGES], (jsv / STAGES) & 1)) {
+                    const int st = jsv % STAGES;
+                    zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jsv), NE, NKB, &S.v_full[st], (jsv / STAGES) & 1);
+                    tc_fence_after();
+                    issue_s(jsv, PE{}, PK{});
+                    if (lane == 0)
+                        umma_commit(&S.s_full[jsv & 1]);
+                    __syncwarp();
+                    ++jsv;
+                    idle = 0;
+                    continue;
+                }
+                if (jpv < jsv && test(&S.p_full[jpv & 1], (jpv >> 1) & 1)) {
+                    issue_pv(jpv);
+                    ++jpv;
+                    idle = 0;
+                    continue;
+                }
+                if (jse < n && jse == jsv && jpv >= jse - 1 && test(&S.e_full[jse % STAGES], (jse / STAGES) & 1)) {
+                    const int st = jse % STAGES;
+                    zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jse), 0, NE, &S.e_full[st], (jse / STAGES) & 1);
+                    tc_fence_after();
+                    issue_s(jse, P0{}, PE{});
+                    if (lane == 0)
+                        umma_commit(&S.e_empty[st]);
+                    __syncwarp();
+                    ++jse;
+                    idle = 0;
+                    continue;
+                }
+                if (++idle >= kWaitLimit)
+                    ok = false;
             }
         }
-        if (ok && n > 0 && !issue_pv(n - 1))
-            ok = false;
         if (!ok && lane == 0)
             raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
         // every MMA this thread issued has completed before TMEM is freed
@@ -391,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[TH / 2];
 #pragma unroll
             for (int i = 0; i < TH / 2; ++i) {
-                const float e0 = exp2f(s[2 * i] - m_use), e1 = exp2f(s[2 * i + 1] - m_use);
+                const float e0 = exp2_approx(s[2 * i] - m_use), e1 = exp2_approx(s[2 * i + 1] - m_use);
                 ps8[i & 7] += e0 + e1;
                 const __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
                 pk[i] = *reinterpret_cast<const uint32_t *>(&v2);

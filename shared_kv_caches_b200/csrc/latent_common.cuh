@@ -13,6 +13,15 @@ constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.f;   // log2 units: O is rescaled only past 2^8
 constexpr int kMaxSplitPages = 1024;       // pages per part the page-validity table holds
 
+// 2^x on the special-function unit (ex2.approx.ftz: ~2 ulp, subnormal results
+// flushed to zero, 2^-inf = 0); the softmax weights are rounded to bf16 next
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
 {
     return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
