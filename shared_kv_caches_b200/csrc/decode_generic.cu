@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kThreads) generic_decode_kernel(const DecodeAr
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x;
+    pdl_launch_dependents();
     const int s = blockIdx.x;
     const int u = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y % a.head_chunks;

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem &S = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+    pdl_launch_dependents();
     const bool mla = !a.mlra && a.NU == 1;
     if (smem_u32(smem_raw) & 1023u) {
         // the 128-byte swizzle atoms need 1024-byte alignment; never expected
@@ -216,32 +217,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 v_issued = 0;
             } else {
-                // E groups may run ahead of V groups: each group waits only for
-                // its own slot; the lower tile goes first when both can
-                uint32_t idle = 0;
-                while (v_issued < n) {
-                    const bool v_can = v_issued < e_issued &&
-                                       (v_issued < STAGES ||
-                                        mbar_test(&S.v_empty[v_issued % STAGES], ((v_issued / STAGES) - 1) & 1));
-                    if (v_can) {
-                        load_group(v_issued, v_issued % STAGES, NE, NKB, &S.v_full[v_issued % STAGES]);
-                        ++v_issued;
-                        idle = 0;
-                        continue;
-                    }
-                    const bool e_can = e_issued < n &&
-                                       (e_issued < STAGES ||
-                                        mbar_test(&S.e_empty[e_issued % STAGES], ((e_issued / STAGES) - 1) & 1));
-                    if (e_can) {
-                        load_group(e_issued, e_issued % STAGES, 0, NE, &S.e_full[e_issued % STAGES]);
-                        ++e_issued;
-                        idle = 0;
-                        continue;
-                    }
-                    if (++idle >= kWaitLimit) {
+                // E(j), then V(j): E(j+1) is not needed before V(j) has landed
+                // (S_{j+1} follows S_j), so the sequence costs nothing, and
+                // the thread sleeps in its waits instead of polling
+                for (int j = 0; j < n; ++j) {
+                    const int st = j % STAGES;
+                    const uint32_t eph = ((j / STAGES) - 1) & 1;
+                    if (j >= STAGES && !mbar_wait(&S.e_empty[st], eph)) {
                         raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
                         break;
                     }
+                    load_group(j, st, 0, NE, &S.e_full[st]);
+                    e_issued = j + 1;
+                    if (j >= STAGES && !mbar_wait(&S.v_empty[st], eph)) {
+                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                        break;
+                    }
+                    load_group(j, st, NE, NKB, &S.v_full[st]);
+                    v_issued = j + 1;
                 }
             }
             // every copy this thread started has landed before the CTA can exit

@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
     MqaSmem &S = *reinterpret_cast<MqaSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    pdl_launch_dependents();
 
     int L = a.seq_lens[b];
     if (L > a.max_seq_len) {

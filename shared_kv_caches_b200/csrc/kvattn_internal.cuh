@@ -60,6 +60,13 @@ struct CombineArgs {
 
 __device__ __forceinline__ void raise_error(int *err, int bit) { atomicOr(err, bit); }
 
+// Programmatic dependent launch: a decode kernel lets the combine pass queued
+// behind it be scheduled at once (its blocks then wait in pdl_wait_primary
+// until every decode CTA has finished and its writes are visible), so the
+// combine's launch overlaps the decode's tail.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Merge of the parts of one (sequence b, rows hu0 .. hu0 + nrows - 1) group,
 // run by the last CTA of the group to finish: lse = ln sum_s exp(lse_s),
 // out = sum_s exp(lse_s - lse) o_s, cast to the output type.  w is shared
