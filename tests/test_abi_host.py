@@ -71,6 +71,35 @@ def test_plan_every_workload(lib, name):
     assert K.kvattn_workspace_size(s.variant_id, p) == plan.workspace_bytes
 
 
+# (kernel, parts, pages per part, CTAs, launches) the planner picks for each
+# benchmark shape at its longest context.  Latent kernels run one CTA per SM:
+# a B=1 problem fills one wave of 148 CTAs (37 parts x 4 branches), larger
+# batches aim at about four waves; GQA aims at four waves of three CTAs per SM
+# and merges its parts in place (one launch); MQA aims at 2.5 waves.
+EXPECTED_PLANS = {
+    "gla": ("latent_tc", 4, 64, 512, 2),
+    "gqa": ("gqa", 7, 19, 1792, 1),
+    "mfa": ("mqa_tc", 12, 11, 384, 2),
+    "mla": ("latent_tc", 5, 103, 640, 2),
+    "mlra_128k": ("latent_tc", 37, 56, 148, 2),
+    "mlra_512k": ("latent_tc", 37, 222, 148, 2),
+    "mlra_1m": ("latent_tc", 37, 444, 148, 2),
+    "mlra_b8_128k": ("latent_tc", 9, 228, 288, 2),
+    "tiny_mla": ("generic", 8, 1, 16, 2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EXPECTED_PLANS))
+def test_plan_of_each_benchmark_shape(lib, name):
+    s, p = _params(name)
+    plan = K.kvattn_get_plan(s.variant_id, p)
+    got = (K.KERNEL_NAMES[plan.kernel], plan.num_splits, plan.pages_per_split, plan.ctas, plan.launches)
+    assert got == EXPECTED_PLANS[name]
+    if name.startswith("mlra"):
+        # whole 128-token tiles per part
+        assert plan.pages_per_split % 2 == 0
+
+
 def test_forced_splits_are_clamped(lib):
     s, p = _params("gqa", num_splits=100000)
     plan = K.kvattn_get_plan(s.variant_id, p)

@@ -240,8 +240,12 @@ def test_context_of_one_returns_value_bits(dev, name):
             np.testing.assert_array_equal(got[b, h], v)
 
 
-def test_page_id_out_of_range_sets_error_and_skips(dev, oracle_mod):
-    shape = SWEEP_SHAPES["gla"].replace(batch=3, ctx=(200, 200))
+@pytest.mark.parametrize("name", ["gla", "mla"])
+def test_page_id_out_of_range_sets_error_and_skips(dev, oracle_mod, name):
+    """A bad page id in one sequence: the error bit is set, that tile loads
+    nothing (both ring groups of the MLA kernel still arrive), and the other
+    sequences are unaffected."""
+    shape = SWEEP_SHAPES[name].replace(batch=3, ctx=(200, 200))
     x = W.make_inputs(shape, seed=8)
     bt = x["block_table"].copy()
     bt[1, 2] = x["num_pages"] + 3          # bad frame id for sequence 1
