@@ -160,7 +160,10 @@ int kvattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
  * (flash-decoding) that sums the MLRA branches, places GLA group heads and
  * casts to out_dtype.  The GQA kernel merges in the last CTA of each
  * (sequence, KV head) to finish (one launch); the others run a combine pass
- * (two launches; kvattn_get_plan reports which).  Returns KVATTN_OK once
+ * (two launches; kvattn_get_plan reports which).  The combine pass is a
+ * programmatic dependent launch of the split pass: the GPU may schedule it
+ * while the split pass drains, and it waits on the device until that pass
+ * has completed and its writes are visible.  Returns KVATTN_OK once
  * enqueued, a negative status (nothing enqueued) for bad arguments,
  * KVATTN_ERR_CUDA if a launch failed.
  */
@@ -174,7 +177,8 @@ int kvattn_decode(int32_t variant, const kvattn_params *p, const void *q_nope, c
  * kernels that merge their own parts this includes the merge), events[2]
  * after the combine pass, or right after events[1] when there is none (a
  * NULL entry is skipped; events may be NULL).  Used to time each pass on the launching
- * stream.  Same arguments, statuses and results as kvattn_decode. */
+ * stream; an event recorded between the passes makes them run strictly one
+ * after the other.  Same arguments, statuses and results as kvattn_decode. */
 int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_nope,
                         const void *q_rope, const void *kv_cache, const int32_t *block_table,
                         const int32_t *seq_lens, float sm_scale, void *out, float *lse,
