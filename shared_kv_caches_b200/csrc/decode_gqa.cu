@@ -1,9 +1,8 @@
-// GQA decode on CUDA cores: 4 query heads per KV head, head dim 128.
+// GQA decode: 4 query heads per KV head, head dim 128.
 //
 // A group of query heads shares one K/V head (MLRA page, GQA bullet), so one
 // CTA owns (part s of the context, KV head, sequence b) and serves the 4 query
-// heads of that KV head from one pass over its pages.  At 4 flop per cache
-// byte the work is HBM-bound and stays on the CUDA cores.
+// heads of that KV head from one pass over its pages.
 //
 // Per CTA: one producer warp streams each 64-token page's K and V tiles of the
 // KV head (2 x 16 KB) into a STAGES-deep shared-memory ring with 3-D TMA loads
@@ -14,12 +13,14 @@
 // states are merged by their max (the same LSE merge the combine pass uses
 // across parts) and the normalised part output and lse go to the workspace.
 //
-// Scores: the 128-wide dot is split over 8 lanes (16 dims each, q held in
-// registers), and the 8 partial sums of 4 heads are reduced with a
-// transposing butterfly (3 shuffle steps leave every lane with one finished
-// (token, head) score).  P.V: every lane owns 4 of the 128 value dims for all
-// 4 heads.  Shared-memory reads of K rows (one 128-byte line per 8 lanes) and
-// V rows (256 bytes per warp) are bank-conflict free under the swizzle.
+// The products run on the tensor cores as warp-level bf16 MMAs (m16n8k16,
+// fp32 accumulate), transposed so that the warp's 16 tokens fill the MMA's 16
+// rows and the 4 heads (padded to 8) its columns: S^T = K Q^T takes the K tile
+// straight from shared memory (ldmatrix) with Q^T held in registers, and
+// O^T = V^T P^T takes V through a transposing ldmatrix and P^T from the score
+// fragments transposed in registers (movmatrix).  On the CUDA cores the bf16
+// unpacking and the per-token reductions around the 16 384 FMAs per token
+// cost more issue slots than the FMAs themselves.
 #include <math.h>
 
 #include "kvattn_internal.cuh"
@@ -43,8 +44,6 @@ constexpr float kLn2 = 0.69314718055994531f;
 struct GqaSmem {
     unsigned char tiles[STAGES][STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
     float ow[CW][G][D];                         // per-warp outputs for the final merge
-    float pw[CW][TPW][G];                       // per-warp probabilities of the current page
-    float aw[CW][G];                            // per-warp rescale factors of the current page
     float mw[CW][G];
     float lw[CW][G];
     uint64_t full[STAGES];
@@ -53,36 +52,52 @@ struct GqaSmem {
     int last;
 };
 
-__device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ float dot8(const float *q, uint4 k)
+// Byte offset of 16-byte chunk c (8 dims) of token row t in a swizzled tile.
+__device__ __forceinline__ uint32_t chunk_off(int t, int c)
 {
-    float s = q[0] * lo16(k.x);
-    s = fmaf(q[1], hi16(k.x), s);
-    s = fmaf(q[2], lo16(k.y), s);
-    s = fmaf(q[3], hi16(k.y), s);
-    s = fmaf(q[4], lo16(k.z), s);
-    s = fmaf(q[5], hi16(k.z), s);
-    s = fmaf(q[6], lo16(k.w), s);
-    s = fmaf(q[7], hi16(k.w), s);
-    return s;
+    return (uint32_t)((c >> 3) * BOX_BYTES + t * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
 
-__device__ __forceinline__ void load_q8(float *dst, const __nv_bfloat16 *src)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
-    const uint4 w = *reinterpret_cast<const uint4 *>(src);
-    dst[0] = lo16(w.x);
-    dst[1] = hi16(w.x);
-    dst[2] = lo16(w.y);
-    dst[3] = hi16(w.y);
-    dst[4] = lo16(w.z);
-    dst[5] = hi16(w.z);
-    dst[6] = lo16(w.w);
-    dst[7] = hi16(w.w);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
 
-__global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_constant__ CUtensorMap kv_map,
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// c (16 x 8, fp32) += a (16 x 16, bf16, row) * b (16 x 8, bf16, col)
+__device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8 x 8 bf16 matrix held one fragment row pair per thread.
+__device__ __forceinline__ uint32_t movm_t(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_constant__ CUtensorMap kv_map,
                                                              const DecodeArgs a)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -143,23 +158,28 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
     }
 
     // ---------------------------------------------------------------- consumers
-    const int g = lane >> 3, j = lane & 7;
-    const int hh = ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);   // head whose score this lane ends with
-    float q0[G][8], q1[G][8];
+    // fragment coordinates: r = row group (token of S^T, dim of O^T, head of
+    // the B operands), c = column pair (heads 2c, 2c+1 of S^T and O^T; only
+    // c < 2 are real heads)
+    const int r = lane >> 2, c = lane & 3;
+    const int mrow = lane & 7, mat = lane >> 3;
+    // Q^T as the B operand of S^T = K Q^T: b0 = dims 16kk + 2c.., b1 = + 8, head r
+    uint32_t qb[D / 16][2];
+    {
+        const __nv_bfloat16 *qr = a.q_nope + ((size_t)b * a.H + kvh * G + (r < G ? r : 0)) * D;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        const __nv_bfloat16 *qr = a.q_nope + ((size_t)b * a.H + kvh * G + h) * D;
-        load_q8(q0[h], qr + 8 * j);
-        load_q8(q1[h], qr + 64 + 8 * j);
+        for (int kk = 0; kk < D / 16; ++kk) {
+            qb[kk][0] = r < G ? *reinterpret_cast<const uint32_t *>(qr + 16 * kk + 2 * c) : 0u;
+            qb[kk][1] = r < G ? *reinterpret_cast<const uint32_t *>(qr + 16 * kk + 8 + 2 * c) : 0u;
+        }
     }
-    float m_run = -INFINITY, l_run = 0.f;
-    float O[G][4];
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2c, 2c+1
+    float o[D / 16][4];                                                 // O^T: dims x heads
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-        O[h][0] = O[h][1] = O[h][2] = O[h][3] = 0.f;
+    for (int mt = 0; mt < D / 16; ++mt)
+        o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
     const int t0 = warp * TPW;
-    const int vbox = lane >> 4, vchunk = (lane & 15) >> 1, vhalf = lane & 1;
     for (int i = 0; i < n; ++i) {
         const int st = i % STAGES;
         if (!mbar_wait(&S.full[st], (i / STAGES) & 1)) {
@@ -170,80 +190,73 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
         const int ntok = min(kPage, L - (p0 + i) * kPage);
         const int nw = S.skip[st] ? 0 : min(max(ntok - t0, 0), TPW);
         if (nw > 0) {
-            const unsigned char *Kb = S.tiles[st];
-            const unsigned char *Vb = Kb + TILE_BYTES;
-            float sc[TPW / 4];
-#pragma unroll
-            for (int it = 0; it < TPW / 4; ++it) {
-                const int t = t0 + 4 * it + g;
-                const int off = t * 128 + ((j ^ (t & 7)) << 4);
-                const uint4 k0 = *reinterpret_cast<const uint4 *>(Kb + off);
-                const uint4 k1 = *reinterpret_cast<const uint4 *>(Kb + BOX_BYTES + off);
-                float part[G];
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-                    part[h] = dot8(q0[h], k0) + dot8(q1[h], k1);
-                // transposing butterfly over the 8 lanes of this token
-                const bool up4 = (lane >> 2) & 1;
-                const float a0 = (up4 ? part[2] : part[0]) +
-                                 __shfl_xor_sync(0xffffffffu, up4 ? part[0] : part[2], 4);
-                const float a1 = (up4 ? part[3] : part[1]) +
-                                 __shfl_xor_sync(0xffffffffu, up4 ? part[1] : part[3], 4);
-                const bool up2 = (lane >> 1) & 1;
-                float c = (up2 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, up2 ? a0 : a1, 2);
-                c += __shfl_xor_sync(0xffffffffu, c, 1);
-                sc[it] = (4 * it + g) < nw ? c * a.scale_log2 : -INFINITY;
+            unsigned char *Kb = S.tiles[st];
+            unsigned char *Vb = Kb + TILE_BYTES;
+            if (nw < TPW) {
+                // value rows of this warp past the context: 0 * NaN would poison the MMA
+                for (int idx = lane; idx < (TPW - nw) * (D / 8); idx += 32)
+                    *reinterpret_cast<uint4 *>(Vb + chunk_off(t0 + nw + idx / (D / 8), idx % (D / 8))) =
+                        make_uint4(0, 0, 0, 0);
+                __syncwarp();
             }
-            // online softmax over this warp's tokens, per head hh
-            float mt = sc[0];
+            const uint32_t kbase = smem_u32(Kb), vbase = smem_u32(Vb);
+            // S^T (16 tokens x 8 head columns) = K Q^T
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int it = 1; it < TPW / 4; ++it)
-                mt = fmaxf(mt, sc[it]);
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-            const float m_new = fmaxf(m_run, mt);
-            const float m_use = m_new == -INFINITY ? 0.f : m_new;
-            const float alpha = exp2f(m_run - m_use);
-            float ps = 0.f;
-#pragma unroll
-            for (int it = 0; it < TPW / 4; ++it) {
-                sc[it] = exp2f(sc[it] - m_use);
-                ps += sc[it];
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(kbase + chunk_off(t0 + ((mat & 1) << 3) + mrow, 2 * kk + (mat >> 1)), a0, a1, a2, a3);
+                mma_bf16(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
             }
-            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-            l_run = l_run * alpha + ps;
-            m_run = m_new;
-            if ((lane & 1) == 0) {
+            // online softmax per head over the warp's tokens (rows r and r + 8)
+            float mx[2];
 #pragma unroll
-                for (int it = 0; it < TPW / 4; ++it)
-                    S.pw[warp][4 * it + g][hh] = sc[it];
-                if (lane < 8)
-                    S.aw[warp][hh] = alpha;
+            for (int e = 0; e < 4; ++e) {
+                const int tok = r + ((e >> 1) << 3);
+                s[e] = tok < nw ? s[e] * a.scale_log2 : -INFINITY;
             }
-            __syncwarp();
-
-            // O = O * alpha + sum_t p_t v_t over this warp's tokens
-            const float4 al = *reinterpret_cast<const float4 *>(S.aw[warp]);
-            const float alv[G] = {al.x, al.y, al.z, al.w};
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    O[h][k] *= alv[h];
-            const unsigned char *vrow = Vb + vbox * BOX_BYTES + vhalf * 8;
-            for (int tl = 0; tl < nw; ++tl) {
-                const int t = t0 + tl;
-                const uint2 v = *reinterpret_cast<const uint2 *>(vrow + t * 128 + ((vchunk ^ (t & 7)) << 4));
-                const float4 p4 = *reinterpret_cast<const float4 *>(S.pw[warp][tl]);
-                const float vv[4] = {lo16(v.x), hi16(v.x), lo16(v.y), hi16(v.y)};
-                const float pp[G] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        O[h][k] = fmaf(pp[h], vv[k], O[h][k]);
+            for (int hh = 0; hh < 2; ++hh) {
+                mx[hh] = fmaxf(s[hh], s[2 + hh]);
+                mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 4));
+                mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 8));
+                mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 16));
             }
+            float alpha[2], m_use[2];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const float m_new = fmaxf(m_run[hh], mx[hh]);
+                m_use[hh] = m_new == -INFINITY ? 0.f : m_new;
+                alpha[hh] = exp2f(m_run[hh] - m_use[hh]);
+                m_run[hh] = m_new;
+            }
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                p[e] = exp2f(s[e] - m_use[e & 1]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float ps = p[hh] + p[2 + hh];
+                ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+                l_run[hh] = l_run[hh] * alpha[hh] + ps;
+            }
+            // P^T as the B operand of O^T = V^T P^T: tokens 2c.. (b0) and 8 + 2c.. (b1) of head r
+            const uint32_t pb0 = movm_t(pack_bf16(p[0], p[1]));
+            const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                o[mt][0] *= alpha[0];
+                o[mt][1] *= alpha[1];
+                o[mt][2] *= alpha[0];
+                o[mt][3] *= alpha[1];
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(vbase + chunk_off(t0 + ((mat >> 1) << 3) + mrow, 2 * mt + (mat & 1)), a0, a1, a2, a3);
+                mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
+            }
+            if (nw < TPW)
+                fence_proxy_async_smem();   // the zeroed rows are rewritten by the next TMA load
         }
         __syncwarp();
         if (lane == 0)
@@ -251,13 +264,20 @@ __global__ void __launch_bounds__(THREADS) gqa_decode_kernel(const __grid_consta
     }
 
     // merge the four warps' states and write this part's result
-    if ((lane & 1) == 0 && lane < 8) {
-        S.mw[warp][hh] = m_run;
-        S.lw[warp][hh] = l_run;
-    }
+    if (c < 2) {
+        if (r == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-        *reinterpret_cast<float4 *>(&S.ow[warp][h][4 * lane]) = make_float4(O[h][0], O[h][1], O[h][2], O[h][3]);
+            for (int hh = 0; hh < 2; ++hh) {
+                S.mw[warp][2 * c + hh] = m_run[hh];
+                S.lw[warp][2 * c + hh] = l_run[hh];
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                S.ow[warp][2 * c + (e & 1)][16 * mt + r + ((e >> 1) << 3)] = o[mt][e];
+    }
     named_sync(1, CW * 32);
 
     const int tid = threadIdx.x;
