@@ -182,6 +182,8 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
                 const int t = ntok + idx / 16, cc = vh * 16 + (idx % 16);
                 *reinterpret_cast<uint4 *>(Vb + chunk_off(t, cc)) = make_uint4(0, 0, 0, 0);
             }
+            // the next TMA load into this stage (async proxy) must land after these stores
+            fence_proxy_async_smem();
             named_sync(2 + vh, 32 * HG);
         }
         if (ntok > 0) {
