@@ -21,23 +21,26 @@
 // columns: two score / probability buffers of T, the output slice, the Q
 // chunks (MLRA 256 + 128 + 96, MLA and GLA 128 + 256 + 128).
 //
-// A stage of the shared-memory ring holds one tile's key boxes in two
-// groups with their own barriers: the E boxes (key columns that are not this
-// slot's values: the rope key, and for MLA the other value half) are free
-// again as soon as the score MMAs that read them complete, the V boxes (this
-// slot's value columns) only after P.V.  The next tiles' E boxes therefore
-// load while a tile's softmax and P.V run, and a V group has the MMAs of a
-// whole tile to land in.
+// MLA's ring is two stages deep (five Q chunks take the rest of shared
+// memory), so its stages hold a tile's key boxes in two groups with their own
+// barriers: the E boxes (key columns that are not this slot's values: the
+// other value half and the rope key) are free again as soon as the score MMAs
+// that read them complete, the V boxes (this slot's value columns) only after
+// P.V.  The next tiles' E boxes therefore load while a tile's softmax and P.V
+// run, and a V group has the MMAs of a whole tile to land in.  GLA and MLRA
+// have four stages and a one-box E group; their stage is one group, freed
+// after P.V.
 //
 // Warp roles (320 threads):
-//   warp 0     TMEM allocation; one thread streams each tile's E group, then
-//              its V group, into a STAGES-deep ring with 2-D TMA loads
-//              (128-byte swizzle; a 128-token tile is two pages)
-//   warp 1     one thread issues the E part of S_j = Q K_j^T into one of two
-//              TMEM score buffers, then, in whichever order their inputs
-//              arrive, the V part of S_j and P_{j-1} V_{j-1} into the TMEM
-//              output; the warp zeroes the rows of a tile past the context
-//              first (0 * NaN would poison the MMA)
+//   warp 0     TMEM allocation; one thread streams the tiles (MLA: each tile's
+//              E group, then its V group) into a STAGES-deep ring with 2-D
+//              TMA loads (128-byte swizzle; a 128-token tile is two pages)
+//   warp 1     one thread issues S_j = Q K_j^T into one of two TMEM score
+//              buffers and P_{j-1} V_{j-1} into the TMEM output: for GLA and
+//              MLRA S_j, then P_{j-1} V_{j-1}; for MLA the E part of S_j,
+//              then the V part of S_j and P_{j-1} V_{j-1} in whichever order
+//              their inputs arrive.  The warp zeroes the rows of a tile past
+//              the context first (0 * NaN would poison the MMA)
 //   warps 2-9  two threads per head row, each owning half of the tile's
 //              columns and half of O's: read S_j from TMEM, exchange the tile
 //              maximum with the partner thread through shared memory, online
