@@ -3,31 +3,37 @@
 
     python bench.py --gpus N --steps K --warmup W [--workload NAME] [--impl reference]
 
-A step is one decode step of the whole path (split pass + combine pass) for
-every problem of the workload over one batch of seeded synthetic input that
-is already resident in HBM.  The default workload is the GQA + MFA pair of the
-benchmark suite: batch 32, 32 query heads, ragged contexts drawn uniformly from
-[1024, 8192] on a paged 64-token bf16 cache with a permuted block table; one
-GQA layer (8 KV heads of 128) and one MFA-style layer (1 KV head of 256) per
-step.  Other workloads (``--workload mla`` etc.) name one problem of
-``shared_kv_caches_b200.workloads.WORKLOADS``.
+The default workload is the whole suite: every decode problem of the
+benchmark (``shared_kv_caches_b200.workloads.WORKLOADS`` minus the tiny parity
+case) is timed in turn, each with its own warm-up and K timed steps.  The
+headline (``value``, ``ms_per_step``, ``roofline``, ``e2e``) is absorbed MLA
+at the DeepSeek-V3 shape (batch 64, 128 query heads, latent 512 + rope 64,
+ragged contexts drawn uniformly from [4096, 32768] on a paged 64-token bf16
+cache with a permuted block table), the largest problem that fits one GPU;
+``suite`` carries the same figures for GQA, MFA, GLA-2 and the four MLRA-4
+shapes.  ``--workload NAME`` times one problem (or ``gqa+mfa``, the GQA and
+MFA layers together as one step).
+
+A step is one decode call of a problem (split pass + combine pass) over one
+batch of seeded synthetic input that is already resident in HBM.
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
 events on the launching stream, with a 252 MiB write between steps (outside
 the events) so every step starts with a cold L2; a barrier and a device
-synchronisation on both sides of the timed loop; the max over ranks is taken.
-With N GPUs every rank runs its own batch (data parallel over sequences, no
-collective on the data path; weak scaling).
+synchronisation on both sides of each timed loop; the max over ranks is
+taken.  With N GPUs every rank runs its own batch (data parallel over
+sequences, no collective on the data path; weak scaling).
 
-The JSON line also carries: the roofline of the dominant kernel (algorithmic
-bytes or flops per launch / its event-timed duration against the measured
-peak), the end-to-end number through the public API with host buffers, the
-oracle timed on the host cores (rank 0, N = 1), SM clocks sampled during the
-timed region, and how many of the library's kernels ran in it.
+The JSON line also carries: the roofline of each problem's decode kernel
+(algorithmic bytes or flops per launch / its event-timed duration against the
+measured peak), the end-to-end number through the public API with host
+buffers, the oracle timed on the host cores for the headline problem (rank 0,
+N = 1), SM clocks sampled during the timed regions, and how many of the
+library's kernels ran in the headline's timed region.
 
-``--impl reference`` times the fp64 CPU oracle (the reference arm) on the same
-workload, each step a bounded sample of it, and prints the same line with
-``"impl": "reference"``.
+``--impl reference`` times the fp64 CPU oracle (the reference arm) on the
+headline problem, each step a bounded sample of it, and prints the same line
+with ``"impl": "reference"``.
 """
 
 from __future__ import annotations
@@ -45,7 +51,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOAD_SETS = {"gqa+mfa": ("gqa", "mfa")}
-DEFAULT_WORKLOAD = "gqa+mfa"
+SUITE = ("mla", "gqa", "mfa", "gla", "mlra_128k", "mlra_512k", "mlra_1m", "mlra_b8_128k")
+DEFAULT_WORKLOAD = "suite"
 METRIC = "decode_attn_tokens_per_s"
 UNIT = "tokens/s"
 
@@ -53,7 +60,7 @@ UNIT = "tokens/s"
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -70,6 +77,9 @@ def parse_args(argv=None):
 
 
 def problem_names(workload):
+    """Problems timed together as one step (the suite's headline is its first)."""
+    if workload == "suite":
+        return SUITE[:1]
     if workload in WORKLOAD_SETS:
         return WORKLOAD_SETS[workload]
     from shared_kv_caches_b200.workloads import WORKLOADS
@@ -133,41 +143,25 @@ def stored_traffic(workload, problem, digest):
 
 # --------------------------------------------------------------------- ours
 
-def run_ours(args, rank, world, local):
+def measure(names, args, dev, world, peaks, flush, workload_label, want_inputs=False):
+    """Time one step (a decode call of every problem in ``names``): W warm-up
+    steps, K event-timed steps with an L2 flush between them, then the same
+    step end to end through the public API.  Returns the figures of the step
+    and of its dominant decode kernel."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     from shared_kv_caches_b200 import benchutil as BU
-    from shared_kv_caches_b200 import build as libbuild
     from shared_kv_caches_b200 import workloads as W
     from shared_kv_caches_b200.device import DeviceProblem
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    if rank == 0:
-        libbuild.build()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-        dist.barrier()
-        if rank != 0:
-            libbuild.build()
-
-    names = problem_names(args.workload)
+    rank = dist_rank()
     seed = BU.rank_seed(args.seed, rank)
     inputs = [W.make_inputs(W.WORKLOADS[n], seed=seed) for n in names]
     probs = [DeviceProblem(x, dev, num_splits=args.splits) for x in inputs]
     costs = [BU.step_cost(x["shape"], x["seq_lens"]) for x in inputs]
     batch = inputs[0]["shape"].batch
-    flush = torch.empty(252 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    peaks = BU.read_peaks(ROOT)
     Ev = torch.cuda.Event
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
 
     def step(evs=None):
         for i, p in enumerate(probs):
@@ -177,9 +171,9 @@ def run_ours(args, rank, world, local):
         step()
         flush.zero_()
     torch.cuda.synchronize()
-    for p in probs:
+    for p, n in zip(probs, names):
         if p.device_error():
-            raise SystemExit(f"device error {p.device_error()} during warm-up")
+            raise SystemExit(f"device error {p.device_error()} during warm-up of {n}")
 
     K = args.steps
     step_ev = [(Ev(enable_timing=True), Ev(enable_timing=True)) for _ in range(K)]
@@ -191,14 +185,8 @@ def run_ours(args, rank, world, local):
             for e in trio:
                 e.record()
     torch.cuda.synchronize()
-    props = torch.cuda.get_device_properties(dev)
-    bus = None
-    if all(hasattr(props, a) for a in ("pci_domain_id", "pci_bus_id", "pci_device_id")):
-        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-    sampler = BU.ClockSampler(bus_id=bus).start()
-    time.sleep(0.3)
 
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     t0 = time.time()
     for k in range(K):
@@ -207,9 +195,11 @@ def run_ours(args, rank, world, local):
         step_ev[k][1].record()
         flush.zero_()
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     t1 = time.time()
-    sampler.stop()
+    for p, n in zip(probs, names):
+        if p.device_error():
+            raise SystemExit(f"device error {p.device_error()} in the timed steps of {n}")
 
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_ms = BU.max_over_ranks(sum(step_ms), dev)
@@ -230,7 +220,7 @@ def run_ours(args, rank, world, local):
     t_mem = c["decode_bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = c["flops"] / (peaks["bf16_tflops"] * 1e12)
     digest = source_digest(probs[dom].plan_kernel_name())
-    traffic = stored_traffic(args.workload, names[dom], digest)
+    traffic = stored_traffic(workload_label, names[dom], digest)
     if t_tc > t_mem:
         achieved = c["flops"] / t_s / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
@@ -244,35 +234,117 @@ def run_ours(args, rank, world, local):
     # a long step): max(memory time, tensor time at the sustained peak) / time
     t_tc_sus = c["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
     roof["frac_sustained"] = round(max(t_mem, t_tc_sus) / t_s, 4)
+    # decode + combine (the whole call) against the binding roof
+    call_s = (decode_ms[dom] + combine_ms[dom]) / 1e3
+    roof["frac_call"] = round(max(t_mem, t_tc) / call_s, 4)
     roof.update({"traffic": traffic, "kernel": f"{names[dom]} decode pass ({probs[dom].plan_kernel_name()})",
                  "algorithmic_bytes": c["decode_bytes"], "algorithmic_flops": c["flops"],
-                 "launch_us": round(decode_ms[dom] * 1e3, 2), "peak_source": peaks["source"] + " (burst)",
-                 "source_digest": digest})
+                 "launch_us": round(decode_ms[dom] * 1e3, 2),
+                 "peak_source": peaks["source"] + " (burst)", "source_digest": digest})
+    if traffic is not None:
+        roof["traffic_per_algorithmic_byte"] = round(traffic / c["decode_bytes"], 3)
 
     total_bytes = sum(x["bytes"] for x in costs)
     total_tokens = sum(x["tokens"] for x in costs) // len(costs)
-    launches = K * sum(p.plan.launches for p in probs)
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(names), "name": args.workload, "batch_per_gpu": batch,
-                   "ctx_tokens_per_gpu": total_tokens, "page_size": 64, "seed": args.seed,
-                   "l2": "flushed between timed steps (252 MiB write outside the events)",
-                   "parallelism": f"dp{world} (independent batches per GPU)"},
+    out = {
+        "names": list(names), "value": round(value, 1), "ms_per_step": round(ms_per_step, 5),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "ctx_tokens_per_s": round(world * total_tokens / (ms_per_step / 1e3), 1),
         "hbm_gbs": round(total_bytes / (ms_per_step / 1e3) / 1e9, 1),
+        "batch": batch, "ctx_tokens": total_tokens, "workload": describe(names),
         "kernels_us": {n: {"decode": round(d * 1e3, 2), "combine": round(cb * 1e3, 2),
-                           "kernel": p.plan_kernel_name(), "splits": int(p.plan.num_splits)}
+                           "kernel": p.plan_kernel_name(), "splits": int(p.plan.num_splits),
+                           "ctas": int(p.plan.ctas)}
                        for n, d, cb, p in zip(names, decode_ms, combine_ms, probs)},
-        "roofline": roof,
-        "e2e": e2e,
-        "gpu_launches": launches,
-        "clocks": sampler.summary(t0, t1),
+        "roofline": roof, "e2e": e2e, "gpu_launches": K * sum(int(p.plan.launches) for p in probs),
+        "window": (t0, t1),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inputs, args.cpu_seconds, batch)
+    if want_inputs:
+        out["inputs"] = inputs
+    del probs
+    torch.cuda.empty_cache()
+    return out
+
+
+def dist_rank():
+    return int(os.environ.get("RANK", "0"))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    from shared_kv_caches_b200 import benchutil as BU
+    from shared_kv_caches_b200 import build as libbuild
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    if rank == 0:
+        libbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+        dist.barrier()
+        if rank != 0:
+            libbuild.build()
+
+    flush = torch.empty(252 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peaks = BU.read_peaks(ROOT)
+    props = torch.cuda.get_device_properties(dev)
+    bus = None
+    if all(hasattr(props, a) for a in ("pci_domain_id", "pci_bus_id", "pci_device_id")):
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    sampler = BU.ClockSampler(bus_id=bus).start()
+    time.sleep(0.3)
+
+    groups = [(n,) for n in SUITE] if args.workload == "suite" else [problem_names(args.workload)]
+    label = (lambda g: g[0]) if args.workload == "suite" else (lambda g: args.workload)
+    cpu = None
+    results = []
+    for gi, g in enumerate(groups):
+        want = gi == 0 and rank == 0 and world == 1 and not args.no_cpu_baseline
+        r = measure(g, args, dev, world, peaks, flush, label(g), want_inputs=want)
+        if want:
+            cpu = cpu_baseline(r.pop("inputs"), args.cpu_seconds, r["batch"])
+        results.append(r)
+    sampler.stop()
+
+    head = results[0]
+    windows = [r["window"] for r in results]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": head["workload"], "name": "+".join(head["names"]),
+                   "batch_per_gpu": head["batch"], "ctx_tokens_per_gpu": head["ctx_tokens"], "page_size": 64,
+                   "seed": args.seed,
+                   "l2": "flushed between timed steps (252 MiB write outside the events)",
+                   "parallelism": f"dp{world} (independent batches per GPU)"},
+        "us_per_step": head["us_per_step"],
+        "ctx_tokens_per_s": head["ctx_tokens_per_s"],
+        "hbm_gbs": head["hbm_gbs"],
+        "kernels_us": head["kernels_us"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": sampler.summary_windows(windows),
+        "clocks_headline": sampler.summary(*head["window"]),
+    }
+    if len(results) > 1:
+        line["suite"] = {
+            "+".join(r["names"]): {k: r[k] for k in ("workload", "value", "us_per_step", "ctx_tokens_per_s",
+                                                     "hbm_gbs", "kernels_us", "roofline", "e2e",
+                                                     "gpu_launches")}
+            for r in results}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

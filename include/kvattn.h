@@ -97,7 +97,8 @@ enum kvattn_device_error {
 /* Which decode kernel a plan uses. */
 enum kvattn_kernel {
     KVATTN_KERNEL_GENERIC = 0,   /* CUDA-core split-KV kernel, any supported shape */
-    KVATTN_KERNEL_GQA = 1,       /* CUDA-core GQA/MQA kernel, bulk-copy staged pages */
+    KVATTN_KERNEL_GQA = 1,       /* GQA kernel: TMA-staged pages, warp-level bf16 MMAs
+                                    (m16n8k16), parts merged in the last CTA of each group */
     KVATTN_KERNEL_LATENT_TC = 2, /* tcgen05/TMEM latent kernel (MLA, GLA, MLRA) */
     KVATTN_KERNEL_MQA_TC = 3     /* tensor-core MQA kernel (one wide KV head) */
 };
@@ -125,7 +126,7 @@ typedef struct {
     int32_t out_dtype;         /* kvattn_out_dtype */
 } kvattn_params;
 
-/* What kvattn_decode will launch for a problem (host only, no CUDA calls). */
+/* What kvattn_decode will launch for a problem (see kvattn_get_plan). */
 typedef struct {
     int32_t kernel;            /* kvattn_kernel */
     int32_t num_splits;        /* parts per context */
@@ -138,7 +139,9 @@ typedef struct {
 } kvattn_plan;
 
 /* Fill *plan for (variant, p).  Returns KVATTN_OK or INVALID_ARG/UNSUPPORTED.
- * Host only; never touches the GPU. */
+ * Host only: no device memory is touched and nothing is enqueued.  The plan is
+ * sized for the current device's SM count, queried once per device through
+ * the CUDA runtime (148, a B200, when no device can be queried). */
 int kvattn_get_plan(int32_t variant, const kvattn_params *p, kvattn_plan *plan);
 
 /* Bytes of workspace kvattn_decode needs for (variant, p): a 256-byte header
@@ -211,16 +214,41 @@ int kvattn_decode_timed(int32_t variant, const kvattn_params *p, const void *q_n
  * KVATTN_ERR_WORKSPACE_TOO_SMALL and enqueues nothing.
  *
  * The first call on a device (that device current) looks up the array's
- * device address; make that first call before any stream capture.  All calls
- * share the one array, which keeps the last call's contents: calls ordered on
- * one stream are safe, calls that overlap on the GPU race on it.  Each call
- * clears the device error word at its start; device_error (device memory, 4
- * bytes, may be NULL) receives that call's kvattn_device_error bits.
+ * device address; make that first call before any stream capture.  Under lazy
+ * module loading (the CUDA default) that first call is also when the array is
+ * reserved on the device, so make it before the caller claims the rest of
+ * HBM.  The address is kept per device and is stale after cudaDeviceReset.
+ * All calls share the one array, which keeps the last call's contents: calls
+ * ordered on one stream are safe, calls that overlap on the GPU race on it.
+ * Arguments are checked as kvattn_decode checks them before anything is
+ * enqueued: a refused call (any negative status) leaves the array untouched.
+ * Each call clears the device error word at its start; device_error (device
+ * memory, 4 bytes, may be NULL) receives that call's kvattn_device_error bits.
  */
 int kvattn_decode_noalloc(int32_t variant, const kvattn_params *p, const void *q_nope,
                           const void *q_rope, const void *kv_cache, const int32_t *block_table,
                           const int32_t *seq_lens, float sm_scale, void *out, float *lse,
                           int32_t *device_error, void *stream);
+
+/*
+ * kvattn_selftest_bounded_wait -- check, on the device, the bounded mbarrier
+ * wait every decode kernel uses.  No page defines it: it tests the library's
+ * own failure detection (a wait that runs out sets
+ * KVATTN_DEVERR_WAIT_TIMEOUT and returns instead of hanging the GPU).
+ *
+ * Enqueues on `stream` one single-warp kernel that initialises two mbarriers,
+ * completes the phase of one of them and then waits, each wait capped at
+ * `tries` attempts (1 <= tries <= 65536): first on the completed phase, which
+ * must succeed, then on the other barrier, which no thread ever arrives on and
+ * must run out.  It ORs into *result (device memory, 4 bytes, caller-zeroed):
+ * KVATTN_DEVERR_WAIT_TIMEOUT when the second wait gave up as it should, and
+ * KVATTN_SELFTEST_MISSED_PHASE when the first wait failed to see a completed
+ * phase.  A correct library leaves exactly KVATTN_DEVERR_WAIT_TIMEOUT.
+ * Returns INVALID_ARG / MISALIGNED for bad arguments (nothing enqueued) and
+ * KVATTN_ERR_CUDA if the launch failed.
+ */
+#define KVATTN_SELFTEST_MISSED_PHASE 256
+int kvattn_selftest_bounded_wait(int32_t *result, int32_t tries, void *stream);
 
 /* Copy the device error word to *code (0 = none, else kvattn_device_error
  * bits).  Synchronises `stream`.  Returns KVATTN_ERR_CUDA if the copy

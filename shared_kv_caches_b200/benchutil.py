@@ -122,8 +122,14 @@ class ClockSampler:
             self._thread.join(timeout=5)
 
     def summary(self, t0: float, t1: float) -> dict:
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        return self.summary_windows([(t0, t1)])
+
+    def summary_windows(self, windows) -> dict:
+        """Median SM clock, max clock and active throttle reasons over the
+        samples inside any of the (t0, t1) windows."""
+        inside = [s for s in self.samples if any(t0 <= s[0] <= t1 for t0, t1 in windows)]
         window = "timed"
+        t0, t1 = min(w[0] for w in windows), max(w[1] for w in windows)
         if len(inside) < 2:
             # the timed region was shorter than the sampling period: take the
             # samples nearest to it

@@ -14,6 +14,8 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr int kMaxDevices = 64;
+
 int validate(int32_t variant, const kvattn_params *p, Problem *pr)
 {
     if (!p || !pr)
@@ -111,6 +113,7 @@ int choose_splits(int forced, long long units, int max_pages, long long target_c
 int make_plan(const Problem &pr, int forced_splits, Plan *pl)
 {
     memset(pl, 0, sizeof *pl);
+    const int num_sms = sm_count();
     const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
     long long base;
     int splits;
@@ -123,14 +126,14 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         // one CTA per SM: for small batches the fewest waves that keep >= 90% of
         // the SMs busy (long parts, little partial-output traffic); several
         // waves to even out ragged large batches
-        long long target = 4LL * kNumSMs;
-        if (base < kNumSMs / 2) {
+        long long target = 4LL * num_sms;
+        if (base < num_sms / 2) {
             for (long long k = 1; k <= 4; ++k) {
-                const long long sp = (k * kNumSMs) / base;
+                const long long sp = (k * num_sms) / base;
                 const long long ctas = sp * base;
-                const long long waves = (ctas + kNumSMs - 1) / kNumSMs;
+                const long long waves = (ctas + num_sms - 1) / num_sms;
                 target = ctas;
-                if (sp >= 1 && ctas * 10 >= waves * kNumSMs * 9)
+                if (sp >= 1 && ctas * 10 >= waves * num_sms * 9)
                     break;
             }
         }
@@ -140,7 +143,7 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunk = 4;
         pl->head_chunks = 1;
         base = (long long)pr.B * pr.NU;
-        splits = choose_splits(forced_splits, base, max_pages, 4LL * 3 * kNumSMs, 4);
+        splits = choose_splits(forced_splits, base, max_pages, 4LL * 3 * num_sms, 4);
     } else if (mqa_mma_supported(pr)) {
         pl->pub.kernel = KVATTN_KERNEL_MQA_TC;
         pl->head_chunk = 32;
@@ -149,7 +152,7 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         // about 2.5 waves of one CTA per SM: measured on 32 x U[1024,8192]
         // contexts, 12 parts decode as fast as 18 and leave the combine a
         // third less to merge (65.8 against 67.5 us per step); 8 parts is slower
-        splits = choose_splits(forced_splits, base, max_pages, 5LL * kNumSMs / 2, 2);
+        splits = choose_splits(forced_splits, base, max_pages, 5LL * num_sms / 2, 2);
     } else {
         const int hc = generic_head_chunk(pr);
         if (!hc)
@@ -160,7 +163,7 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunk = hc;
         pl->head_chunks = pr.HPU / hc;
         base = (long long)pr.B * pr.NU * pl->head_chunks;
-        splits = choose_splits(forced_splits, base, max_pages, 2LL * kNumSMs, 1);
+        splits = choose_splits(forced_splits, base, max_pages, 2LL * num_sms, 1);
     }
     int pps = (max_pages + splits - 1) / splits;
     if (pl->pub.kernel == KVATTN_KERNEL_LATENT_TC) {
@@ -190,6 +193,47 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
 }
 
 }  // namespace
+
+int sm_count()
+{
+    static int cached[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();   // a failed query leaves its error as the last error: clear it
+        return kDefaultSMs;
+    }
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return kDefaultSMs;
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
+                  const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
+                  float sm_scale, const void *out, const float *lse, const void *workspace,
+                  Problem *pr)
+{
+    int st = validate(variant, p, pr);
+    if (st)
+        return st;
+    if (!q_nope || !kv_cache || !seq_lens || !out || !workspace)
+        return KVATTN_ERR_INVALID_ARG;
+    if (pr->dr > 0 && !q_rope)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!isfinite(sm_scale))
+        return KVATTN_ERR_INVALID_ARG;
+    if (!aligned(q_nope, 16) || (q_rope && !aligned(q_rope, 16)) || !aligned(kv_cache, 16) ||
+        !aligned(out, 16) || (lse && !aligned(lse, 4)) || !aligned(workspace, 256) ||
+        !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
+        return KVATTN_ERR_MISALIGNED;
+    return KVATTN_OK;
+}
+
 }  // namespace kvattn
 
 using namespace kvattn;
@@ -255,19 +299,10 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
                                    size_t workspace_bytes, void *stream, void *const *events)
 {
     Problem pr;
-    int st = validate(variant, p, &pr);
+    int st = validate_call(variant, p, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale, out,
+                           lse, workspace, &pr);
     if (st)
         return st;
-    if (!q_nope || !kv_cache || !seq_lens || !out || !workspace)
-        return KVATTN_ERR_INVALID_ARG;
-    if (pr.dr > 0 && !q_rope)
-        return KVATTN_ERR_INVALID_ARG;
-    if (!isfinite(sm_scale))
-        return KVATTN_ERR_INVALID_ARG;
-    if (!aligned(q_nope, 16) || (q_rope && !aligned(q_rope, 16)) || !aligned(kv_cache, 16) ||
-        !aligned(out, 16) || (lse && !aligned(lse, 4)) || !aligned(workspace, 256) ||
-        !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
-        return KVATTN_ERR_MISALIGNED;
     Plan pl;
     st = make_plan(pr, p->num_splits, &pl);
     if (st)

@@ -266,11 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // zero rows [ntok, T) of stage positions [p_lo, p_hi) once the group's
         // copies (whole boxes, rows past the context included) have landed;
-        // every lane observes the completed phase before it writes
-        auto zero_tail = [&](int st, int ntok, int p_lo, int p_hi, uint64_t *full, uint32_t parity) {
+        // every lane observes the completed phase before it writes.  False
+        // (nothing written) if a lane's wait ran out.
+        auto zero_tail = [&](int st, int ntok, int p_lo, int p_hi, uint64_t *full, uint32_t parity) -> bool {
             if (ntok >= T)
-                return;
-            mbar_wait(full, parity);
+                return true;
+            if (!__all_sync(0xffffffffu, mbar_wait(full, parity)))
+                return false;
             const int rows = T - ntok, nb = p_hi - p_lo;
             for (int idx = lane; idx < rows * nb * 8; idx += 32) {
                 const int box = p_lo + idx / (rows * 8), rem = idx % (rows * 8);
@@ -280,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
+            return true;
         };
         // Descriptors are built once; a byte offset moves the start-address
         // field by offset >> 4 (shared addresses stay below 256 KB, so the
@@ -339,7 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, j), 0, NKB, &S.e_full[st], fph);
+                if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, j), 0, NKB, &S.e_full[st], fph)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 issue_s(j, P0{}, PK{});
                 if (lane == 0)
@@ -372,7 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (ok && jpv < n) {
                 if (jsv < jse && test(&S.v_full[jsv % STAGES], (jsv / STAGES) & 1)) {
                     const int st = jsv % STAGES;
-                    zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jsv), NE, NKB, &S.v_full[st], (jsv / STAGES) & 1);
+                    if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jsv), NE, NKB, &S.v_full[st], (jsv / STAGES) & 1)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     issue_s(jsv, PE{}, PK{});
                     if (lane == 0)
@@ -390,7 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (jse < n && jse == jsv && jpv >= jse - 1 && test(&S.e_full[jse % STAGES], (jse / STAGES) & 1)) {
                     const int st = jse % STAGES;
-                    zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jse), 0, NE, &S.e_full[st], (jse / STAGES) & 1);
+                    if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jse), 0, NE, &S.e_full[st], (jse / STAGES) & 1)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     issue_s(jse, P0{}, PE{});
                     if (lane == 0)

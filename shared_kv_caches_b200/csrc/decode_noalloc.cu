@@ -14,9 +14,13 @@
 // Set-up: the first call on a device, with that device current, looks up the
 // array's device address with cudaGetSymbolAddress (in host code the array's
 // name is only a host-side stand-in, not a device address) and keeps it for
-// that device.  Make that first call before any stream capture.  No call
-// allocates: there is no cudaMalloc, cudaFree or allocating library routine on
-// this path.  All calls share the one array and it keeps the last call's
+// that device.  Make that first call before any stream capture.  With lazy
+// module loading (the CUDA default since 12.2) that same first call is also
+// when the driver loads this code onto the device and reserves the array, so
+// make it before the caller takes the rest of HBM for itself.  The cached
+// address is stale after cudaDeviceReset; the library does not notice a reset.
+// No call allocates: there is no cudaMalloc, cudaFree or allocating library
+// routine on this path.  All calls share the one array and it keeps the last call's
 // contents, so calls that overlap on the GPU (different streams, no ordering
 // between them) race on it; calls on one stream are ordered and safe.
 #include <mutex>
@@ -89,6 +93,13 @@ extern "C" int kvattn_decode_noalloc(int32_t variant, const kvattn_params *p, co
     }
     void *scratch = nullptr;
     st = scratch_for_current_device(&scratch);
+    if (st)
+        return st;
+    // every argument check kvattn_decode makes, before the scratch is touched,
+    // so that a refused call enqueues nothing
+    Problem pr;
+    st = validate_call(variant, &q, q_nope, q_rope, kv_cache, block_table, seq_lens, sm_scale, out, lse,
+                       scratch, &pr);
     if (st)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -12,7 +12,7 @@
 namespace kvattn {
 
 constexpr int kPage = 64;               // tokens per cache page
-constexpr int kNumSMs = 148;            // B200 streaming multiprocessors
+constexpr int kDefaultSMs = 148;        // B200; used when no device can be queried
 constexpr size_t kWsHeader = 256;       // workspace header: device error word
 constexpr int kMaxSplits = 1024;
 
@@ -147,6 +147,18 @@ __device__ __forceinline__ bool finish_part(const DecodeArgs &a, int ticket_idx,
     }
     return last;
 }
+
+// Streaming multiprocessors of the current device (queried once per device
+// through the runtime; kDefaultSMs when there is no device).
+int sm_count();
+
+// Argument checks shared by every decode entry point: the problem, the
+// pointers and their alignment, sm_scale.  Returns a kvattn_status; nothing
+// is enqueued.
+int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
+                  const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
+                  float sm_scale, const void *out, const float *lse, const void *workspace,
+                  Problem *pr);
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_generic(const DecodeArgs &a, int head_chunk, cudaStream_t st);

@@ -32,10 +32,11 @@ KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1
 KVATTN_DEVERR_SEQ_TOO_LONG = 2
 KVATTN_DEVERR_WAIT_TIMEOUT = 4
 KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc"}
+KVATTN_SELFTEST_MISSED_PHASE = 256
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
            "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
-           "kvattn_status_string", "kvattn_version")
+           "kvattn_status_string", "kvattn_version", "kvattn_selftest_bounded_wait")
 KVATTN_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -83,9 +84,10 @@ def load():
     lib.kvattn_status_string.argtypes = [ctypes.c_int]
     lib.kvattn_status_string.restype = ctypes.c_char_p
     lib.kvattn_version.argtypes = []
+    lib.kvattn_selftest_bounded_wait.argtypes = [vp, i32, vp]
     for name in ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
                  "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
-                 "kvattn_version"):
+                 "kvattn_version", "kvattn_selftest_bounded_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -150,6 +152,11 @@ def kvattn_decode_noalloc(variant, params, q_nope, q_rope, kv_cache, block_table
     return load().kvattn_decode_noalloc(int(variant), ctypes.byref(params), q_nope, q_rope, kv_cache,
                                         block_table, seq_lens, float(sm_scale), out, lse, device_error,
                                         stream)
+
+
+def kvattn_selftest_bounded_wait(result: int, tries: int, stream: int = 0) -> int:
+    """Enqueue the bounded-wait self-test; returns its status."""
+    return load().kvattn_selftest_bounded_wait(result, int(tries), stream)
 
 
 def kvattn_get_device_error(workspace: int, stream: int = 0) -> int:

@@ -160,10 +160,15 @@ WORKLOADS = {
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 to bf16 (round to nearest, ties to even); finite inputs."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = u + 0x7FFF + ((u >> 16) & 1)
-    return (u >> 16).astype(np.uint16)
+    """Round float32 to bf16 (round to nearest, ties to even); finite inputs.
+
+    In 32-bit arithmetic: a finite float's bits plus at most 0x8000 stay below
+    2**32, so nothing wraps."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    v = (u >> 16) & 1
+    v += u
+    v += 0x7FFF
+    return (v >> 16).astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -37,3 +37,26 @@ def test_stored_traffic_matches_only_current_digest():
         assert bench.stored_traffic(wl, prob, digest) == float(nbytes)
         assert bench.stored_traffic(wl, prob, "0" * 16) is None
     assert bench.stored_traffic("no-such-workload", "x", rows[0][4]) is None
+
+
+def test_suite_covers_every_benchmark_problem():
+    """The default run times every benchmark problem except the tiny parity
+    case, with MLA (the largest single-GPU problem) as the headline."""
+    from shared_kv_caches_b200 import workloads as W
+    assert bench.DEFAULT_WORKLOAD == "suite"
+    assert set(bench.SUITE) == set(W.WORKLOADS) - {"tiny_mla"}
+    assert bench.SUITE[0] == "mla"
+    assert bench.problem_names("suite") == ("mla",)
+    assert bench.problem_names("gqa+mfa") == ("gqa", "mfa")
+
+
+def test_clock_summary_over_several_windows():
+    from shared_kv_caches_b200.benchutil import ClockSampler
+    cs = ClockSampler()
+    none = {r: False for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")}
+    cap = dict(none, sw_power_cap=True)
+    cs.samples = [(1.0, 1965.0, 1965.0, 500.0, none), (2.0, 1900.0, 1965.0, 900.0, cap),
+                  (5.0, 1000.0, 1965.0, 100.0, none), (8.0, 1965.0, 1965.0, 600.0, none)]
+    s = cs.summary_windows([(0.5, 2.5), (7.5, 8.5)])
+    assert s["samples"] == 3 and s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] == 1965.0
+    assert cs.summary(4.0, 6.0)["window"] == "nearest"

@@ -5,9 +5,11 @@ plugin host that passes only inputs and outputs, a path where a cudaMalloc's
 possible device synchronisation is not acceptable) get an entry point whose
 scratch is a fixed device array inside the library.  These tests call it
 through the C ABI twice in a row, on two different problems, and compare each
-result with kvattn_decode's within the parity tolerances; they also check that
-a problem too large for the array is refused and that the per-call device
-error word is reported and cleared.  This file is collected last on purpose.
+result with kvattn_decode's within the parity tolerances and with the fp64
+oracle; they also run a problem that fits the array only with fewer parts per
+context than the library would choose, check that a problem too large for the
+array is refused, and that the per-call device error word is reported and
+cleared.  This file is collected last on purpose.
 """
 
 import numpy as np
@@ -51,7 +53,7 @@ def _close(a_out, a_lse, b_out, b_lse):
     assert err <= TOL_MAX and rel <= TOL_REL and dl <= TOL_LSE, (err, rel, dl)
 
 
-def test_two_calls_in_a_row_match_kvattn_decode(dev):
+def test_two_calls_in_a_row_match_kvattn_decode(dev, oracle_mod):
     import torch
     from shared_kv_caches_b200.device import DeviceProblem
     shapes = [W.WORKLOADS["gqa"].replace(batch=4, ctx=(1, 3000)),
@@ -70,6 +72,62 @@ def test_two_calls_in_a_row_match_kvattn_decode(dev):
         out, lse = p.results()
         _close(out, lse, ref_out, ref_lse)
         assert int(err.item()) == 0
+        orc_out, orc_lse = oracle_mod.decode(x)
+        _close(out, lse, orc_out, orc_lse)
+
+
+def test_problem_that_fits_only_with_fewer_parts(dev, oracle_mod):
+    """The library's own plan for this MLA batch needs more scratch than the
+    array holds; the entry point lowers the part count until it fits and
+    must then give kvattn_decode's result for that part count."""
+    import torch
+    from shared_kv_caches_b200.device import DeviceProblem
+    shape = W.WORKLOADS["mla"].replace(batch=64, ctx=(8192, 8192))
+    x = W.make_inputs(shape, seed=41)
+    params = K.params_for(shape, x["max_pages_per_seq"], x["num_pages"], 8192)
+    auto = K.kvattn_get_plan(K.KVATTN_MLA, params)
+    assert auto.workspace_bytes > K.KVATTN_NOALLOC_SCRATCH_BYTES, auto.workspace_bytes
+    fit = None
+    for s in range(auto.num_splits - 1, 0, -1):
+        q = K.params_for(shape, x["max_pages_per_seq"], x["num_pages"], 8192, num_splits=s)
+        if K.kvattn_get_plan(K.KVATTN_MLA, q).workspace_bytes <= K.KVATTN_NOALLOC_SCRATCH_BYTES:
+            fit = s
+            break
+    assert fit is not None
+    p = DeviceProblem(x, dev, num_splits=fit)
+    p.run()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = p.results()
+    p.params = params                        # the caller's request: library choice of parts
+    p.out.fill_(float("nan"))
+    p.lse.fill_(float("nan"))
+    err = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    assert _noalloc(p, err) == K.KVATTN_OK
+    torch.cuda.synchronize()
+    out, lse = p.results()
+    _close(out, lse, ref_out, ref_lse)
+    assert int(err.item()) == 0
+    b_list = [0, 37, 63]
+    orc_out, orc_lse = oracle_mod.decode(x, b_list=b_list)
+    _close(out[b_list], lse[b_list], orc_out, orc_lse)
+
+
+def test_refused_call_leaves_the_array_alone(dev):
+    """A call refused for a bad pointer enqueues nothing (the next good call
+    still reports only its own errors)."""
+    import torch
+    from shared_kv_caches_b200.device import DeviceProblem
+    x = W.make_inputs(W.WORKLOADS["gla"].replace(batch=1, ctx=(100, 100)), seed=42)
+    p = DeviceProblem(x, dev)
+    st = K.kvattn_decode_noalloc(p.variant, p.params, p.q_nope.data_ptr() + 2, p.q_rope.data_ptr(),
+                                 p.kv.data_ptr(), p.block_table.data_ptr(), p.seq_lens.data_ptr(),
+                                 p.sm_scale, p.out.data_ptr(), p.lse.data_ptr(), None,
+                                 torch.cuda.current_stream(dev).cuda_stream)
+    assert st == K.KVATTN_ERR_MISALIGNED
+    st = K.kvattn_decode_noalloc(p.variant, p.params, p.q_nope.data_ptr(), p.q_rope.data_ptr(),
+                                 p.kv.data_ptr(), p.block_table.data_ptr(), None, p.sm_scale,
+                                 p.out.data_ptr(), p.lse.data_ptr(), None, 0)
+    assert st == K.KVATTN_ERR_INVALID_ARG
 
 
 def test_noalloc_reports_and_clears_device_errors(dev):
