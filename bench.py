@@ -109,6 +109,7 @@ KERNEL_SOURCES = {
     "gqa": ["decode_gqa.cu"],
     "mqa_tc": ["decode_mqa_mma.cu"],
     "latent_tc": ["decode_latent_tc.cu", "latent_common.cuh"],
+    "latent_pair": ["decode_mla_pair.cu", "latent_common.cuh"],
     "generic": ["decode_generic.cu"],
 }
 SHARED_SOURCES = ["kvattn_internal.cuh", "sm100.cuh"]

@@ -99,8 +99,12 @@ enum kvattn_kernel {
     KVATTN_KERNEL_GENERIC = 0,   /* CUDA-core split-KV kernel, any supported shape */
     KVATTN_KERNEL_GQA = 1,       /* GQA kernel: TMA-staged pages, warp-level bf16 MMAs
                                     (m16n8k16), parts merged in the last CTA of each group */
-    KVATTN_KERNEL_LATENT_TC = 2, /* tcgen05/TMEM latent kernel (MLA, GLA, MLRA) */
-    KVATTN_KERNEL_MQA_TC = 3     /* tensor-core MQA kernel (one wide KV head) */
+    KVATTN_KERNEL_LATENT_TC = 2, /* tcgen05/TMEM latent kernel, one CTA per group or branch
+                                    (GLA, MLRA) */
+    KVATTN_KERNEL_MQA_TC = 3,    /* tensor-core MQA kernel (one wide KV head) */
+    KVATTN_KERNEL_LATENT_PAIR = 4 /* tcgen05/TMEM MLA kernel (512 + 64) on a 2-CTA cluster:
+                                     each CTA scores half of every page and keeps half of
+                                     the value columns */
 };
 
 /*

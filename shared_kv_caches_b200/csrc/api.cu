@@ -117,9 +117,10 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
     const int max_pages = pr.max_seq_len > 0 ? (pr.max_seq_len + kPage - 1) / kPage : 1;
     long long base;
     int splits;
-    const int tc_slots = latent_tc_slots(pr);
+    const bool pair = latent_pair_supported(pr);
+    const int tc_slots = pair ? 2 : latent_tc_slots(pr);
     if (tc_slots > 0) {
-        pl->pub.kernel = KVATTN_KERNEL_LATENT_TC;
+        pl->pub.kernel = pair ? KVATTN_KERNEL_LATENT_PAIR : KVATTN_KERNEL_LATENT_TC;
         pl->head_chunk = 128;
         pl->head_chunks = tc_slots;
         base = (long long)pr.B * tc_slots;
@@ -166,9 +167,9 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         splits = choose_splits(forced_splits, base, max_pages, 2LL * num_sms, 1);
     }
     int pps = (max_pages + splits - 1) / splits;
-    if (pl->pub.kernel == KVATTN_KERNEL_LATENT_TC) {
+    if (pl->pub.kernel == KVATTN_KERNEL_LATENT_TC || pl->pub.kernel == KVATTN_KERNEL_LATENT_PAIR) {
         // whole tiles per part, and no more pages than the kernel's page table holds
-        const int m = latent_tc_page_multiple(pr);
+        const int m = pl->pub.kernel == KVATTN_KERNEL_LATENT_PAIR ? 1 : latent_tc_page_multiple(pr);
         const int cap = latent_tc_max_pages_per_split();
         pps = (pps + m - 1) / m * m;
         if (pps > cap)
@@ -354,6 +355,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     case KVATTN_KERNEL_GQA: le = launch_gqa(a, s); break;
     case KVATTN_KERNEL_MQA_TC: le = launch_mqa_mma(a, s); break;
     case KVATTN_KERNEL_LATENT_TC: le = launch_latent_tc(a, pr, s); break;
+    case KVATTN_KERNEL_LATENT_PAIR: le = launch_latent_pair(a, s); break;
     default: le = launch_generic(a, pl.head_chunk, s); break;
     }
     if (le != cudaSuccess)

@@ -168,6 +168,8 @@ bool gqa_supported(const Problem &pr);
 cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st);
 bool mqa_mma_supported(const Problem &pr);
 cudaError_t launch_mqa_mma(const DecodeArgs &a, cudaStream_t st);
+bool latent_pair_supported(const Problem &pr);
+cudaError_t launch_latent_pair(const DecodeArgs &a, cudaStream_t st);
 int latent_tc_slots(const Problem &pr);
 int latent_tc_page_multiple(const Problem &pr);
 int latent_tc_max_pages_per_split();

@@ -314,10 +314,64 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank)
     return r;
 }
 
-__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float a, float b, float c, float d)
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v)
 {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32x4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
+}
+
+// Store a float into another CTA's shared memory and count its 4 bytes on an
+// mbarrier there (complete_tx): the consumer waits on its own barrier, no
+// fence or release is needed on this side.
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(remote_addr), "f"(v),
+                 "r"(remote_bar)
+                 : "memory");
+}
+
+// Store 16 bytes into another CTA's shared memory, counted on an mbarrier there.
+__device__ __forceinline__ void st_async_u32x4(uint32_t remote_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                               uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     remote_addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
+                 : "memory");
+}
+
+// Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from this
+// CTA's shared memory into another CTA's, counted on an mbarrier there.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, const void *src, uint32_t bytes,
+                                                  uint32_t remote_bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     remote_dst),
+                 "r"(smem_u32(src)), "r"(bytes), "r"(remote_bar)
+                 : "memory");
+}
+
+// Order this thread's generic-proxy writes to shared memory anywhere in the
+// cluster before later async-proxy reads of it (a peer's tcgen05.mma).
+__device__ __forceinline__ void fence_proxy_async_cluster()
+{
+    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
+// Arrive on the mbarrier at the same shared-memory offset in every CTA of
+// cta_mask once this thread's earlier tcgen05 operations have completed.
+__device__ __forceinline__ void umma_commit_multicast(uint64_t *bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // Arrive on an mbarrier of another CTA in the cluster (release at cluster scope).
@@ -339,9 +393,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 }
 
 // Bounded wait with cluster-scope acquire (data written by the other CTA).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t limit = kWaitLimit)
 {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
+    for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait_cluster(bar, parity))
             return true;
     return false;

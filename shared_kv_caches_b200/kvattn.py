@@ -31,7 +31,7 @@ KVATTN_ERR_CUDA = -5
 KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1
 KVATTN_DEVERR_SEQ_TOO_LONG = 2
 KVATTN_DEVERR_WAIT_TIMEOUT = 4
-KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc"}
+KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc", 4: "latent_pair"}
 KVATTN_SELFTEST_MISSED_PHASE = 256
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",

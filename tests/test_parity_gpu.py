@@ -144,7 +144,8 @@ def test_benchmark_shapes_use_the_specialised_kernels(dev):
     """The benchmark shapes run on their specialised kernels, not the generic one."""
     assert kernel_of(W.WORKLOADS["gqa"]) == "gqa"
     assert kernel_of(W.WORKLOADS["mfa"]) == "mqa_tc"
-    for n in ("mla", "gla", "mlra_128k", "mlra_1m", "mlra_b8_128k"):
+    assert kernel_of(W.WORKLOADS["mla"]) == "latent_pair"
+    for n in ("gla", "mlra_128k", "mlra_1m", "mlra_b8_128k"):
         assert kernel_of(W.WORKLOADS[n]) == "latent_tc", n
     assert kernel_of(W.WORKLOADS["tiny_mla"]) == "generic"
 
