@@ -498,6 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             tc_fence_after();
             const uint32_t s_addr = tS + lane_addr + sb * T + half * TH;
+            // raw scores: the scale is folded into the exponent's FMA, and the
+            // tile maximum of c * s is c times the maximum (for a negative
+            // scale the minimum) of the raw scores
+            const float c = a.scale_log2;
             float s[TH];
             {
                 uint32_t r[TH];
@@ -509,24 +513,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld16(s_addr, r);
 #pragma unroll
                 for (int i = 0; i < TH; ++i)
-                    s[i] = __uint_as_float(r[i]) * a.scale_log2;
+                    s[i] = __uint_as_float(r[i]);
             }
             const int ntok = tile_ntok<T>(S.pvalid, L, p0, j);
-            if (ntok < T) {
+            const int nvalid = ntok - half * TH;                 // valid columns of this thread
+            const bool partial = nvalid < TH;
+            float mt;
+            if (c >= 0.f) {
+                if (partial) {
 #pragma unroll
-                for (int i = 0; i < TH; ++i)
-                    s[i] = half * TH + i < ntok ? s[i] : -INFINITY;
+                    for (int i = 0; i < TH; ++i)
+                        s[i] = i < nvalid ? s[i] : -INFINITY;
+                }
+                const float e = reduce_extreme<true, TH>(s);
+                mt = e == -INFINITY ? -INFINITY : c * e;
+            } else {
+                if (partial) {
+#pragma unroll
+                    for (int i = 0; i < TH; ++i)
+                        s[i] = i < nvalid ? s[i] : INFINITY;
+                }
+                const float e = reduce_extreme<false, TH>(s);
+                mt = e == INFINITY ? -INFINITY : c * e;
             }
-            float mx8[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                mx8[q] = s[q];
-#pragma unroll
-                for (int i = q + 8; i < TH; i += 8)
-                    mx8[q] = fmaxf(mx8[q], s[i]);
-            }
-            float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             // the row max over both halves: swap through shared memory with the
             // partner warp (bounded wait on the quarter's exchange barrier)
             S.xmax[sb][half][h] = mt;
@@ -545,17 +554,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 m_ref = mt;
             }
-            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-            float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
+            float sx[4] = {0.f, 0.f, 0.f, 0.f}, sy[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pk[TH / 2];
 #pragma unroll
             for (int i = 0; i < TH / 2; ++i) {
-                const float e0 = exp2_approx(s[2 * i] - m_use), e1 = exp2_approx(s[2 * i + 1] - m_use);
-                ps8[i & 7] += e0 + e1;
+                float x0, x1;
+                ffma2(x0, x1, s[2 * i], s[2 * i + 1], c, c, nm, nm);
+                if (partial) {
+                    x0 = 2 * i < nvalid ? x0 : -INFINITY;
+                    x1 = 2 * i + 1 < nvalid ? x1 : -INFINITY;
+                }
+                const float e0 = exp2_approx(x0), e1 = exp2_approx(x1);
+                fadd2(sx[i & 3], sy[i & 3], sx[i & 3], sy[i & 3], e0, e1);
                 const __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
                 pk[i] = *reinterpret_cast<const uint32_t *>(&v2);
             }
-            const float ps = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+            const float ps = ((sx[0] + sy[0]) + (sx[1] + sy[1])) + ((sx[2] + sy[2]) + (sx[3] + sy[3]));
             l = l * alpha + ps;
             // P (bf16 pairs) over this half's columns of the score buffer
             const uint32_t p_addr = tS + lane_addr + sb * T + half * (TH / 2);

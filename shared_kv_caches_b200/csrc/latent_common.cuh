@@ -22,6 +22,62 @@ __device__ __forceinline__ float exp2_approx(float x)
     return y;
 }
 
+// d = a * b + c on two fp32 lanes at once (one packed FMA instruction)
+__device__ __forceinline__ void ffma2(float &dx, float &dy, float ax, float ay, float bx, float by, float cx, float cy)
+{
+    asm("{\n\t.reg .b64 a2, b2, c2, d2;\n\tmov.b64 a2, {%2, %3};\n\tmov.b64 b2, {%4, %5};\n\tmov.b64 c2, {%6, %7};\n\t"
+        "fma.rn.f32x2 d2, a2, b2, c2;\n\tmov.b64 {%0, %1}, d2;\n\t}"
+        : "=f"(dx), "=f"(dy)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by), "f"(cx), "f"(cy));
+}
+
+// d = a + b on two fp32 lanes at once
+__device__ __forceinline__ void fadd2(float &dx, float &dy, float ax, float ay, float bx, float by)
+{
+    asm("{\n\t.reg .b64 a2, b2, d2;\n\tmov.b64 a2, {%2, %3};\n\tmov.b64 b2, {%4, %5};\n\t"
+        "add.rn.f32x2 d2, a2, b2;\n\tmov.b64 {%0, %1}, d2;\n\t}"
+        : "=f"(dx), "=f"(dy)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+}
+
+// three-input maximum and minimum
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Maximum (kMax) or minimum of n values, n a multiple of 8.
+template <bool kMax, int n>
+__device__ __forceinline__ float reduce_extreme(const float *v)
+{
+    static_assert(n % 8 == 0, "multiple of 8");
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        acc[q] = v[q];
+#pragma unroll
+        for (int i = q + 8; i < n; i += 16) {
+            if (i + 8 < n)
+                acc[q] = kMax ? fmax3(acc[q], v[i], v[i + 8]) : fmin3(acc[q], v[i], v[i + 8]);
+            else
+                acc[q] = kMax ? fmaxf(acc[q], v[i]) : fminf(acc[q], v[i]);
+        }
+    }
+    const float x = kMax ? fmax3(acc[0], acc[1], acc[2]) : fmin3(acc[0], acc[1], acc[2]);
+    const float y = kMax ? fmax3(acc[3], acc[4], acc[5]) : fmin3(acc[3], acc[4], acc[5]);
+    const float z = kMax ? fmaxf(acc[6], acc[7]) : fminf(acc[6], acc[7]);
+    return kMax ? fmax3(x, y, z) : fmin3(x, y, z);
+}
+
 __device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
 {
     return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
