@@ -1,46 +1,31 @@
-// Latent decode on the 5th-generation tensor cores: absorbed MLA, GLA and
-// MLRA.
+// Latent decode on the 5th-generation tensor cores: GLA and MLRA (and their
+// single-group or single-branch shards).
 //
-// Every query head scores the same cached latent rows (MLRA page: after
-// absorption MLA decodes as one 576-wide MQA head; GLA page: one latent head
-// per query group; MLRA page: the latent split into branches attended on
-// their own), so the scores and P.V are real [128 heads x K] x [K x tokens]
-// contractions and run as tcgen05 MMAs with fp32 accumulators in TMEM.
+// Every query head scores the same cached latent rows (GLA page: one latent
+// head per query group; MLRA page: the latent split into branches attended on
+// their own, branch outputs summed afterwards), so the scores and P.V are real
+// [heads x K] x [K x tokens] contractions and run as tcgen05 MMAs with fp32
+// accumulators in TMEM.  (Absorbed MLA, one 512-wide latent, runs on the
+// 2-CTA kernel in decode_mla_pair.cu.)
 //
-// One CTA owns (part s of the context, slot, sequence b).  A slot is a value
-// half for MLA (the 128 x 512 fp32 output would fill all 512 TMEM columns, so
-// two CTAs each keep 256 value columns and both form the full scores), a
-// latent group for GLA (its 64 heads padded to the MMA's 128 rows) and a
-// branch for MLRA.  Key columns of the slot are [latent slice | shared rope
-// key], each a 64-column box of the page row.
+// One CTA owns (part s of the context, slot, sequence b).  A slot is a latent
+// group for GLA (its heads padded to the MMA's 128 rows) and a branch for
+// MLRA (all heads, each with its own query slice).  Key columns of the slot
+// are [latent slice | shared rope key], each a 64-column box of the page row.
 //
 // The query rows are the MMA's A operand for every tile.  Their first NQT
 // 64-column chunks sit in TMEM (an A operand in TMEM costs no shared-memory
-// bandwidth; with a narrow score tile the re-read of a 128-row A from shared
-// memory would otherwise bound the MMA), the rest in shared memory.  TMEM
-// columns: two score / probability buffers of T, the output slice, the Q
-// chunks (MLRA 256 + 128 + 96, MLA and GLA 128 + 256 + 128).
-//
-// MLA's ring is two stages deep (five Q chunks take the rest of shared
-// memory), so its stages hold a tile's key boxes in two groups with their own
-// barriers: the E boxes (key columns that are not this slot's values: the
-// other value half and the rope key) are free again as soon as the score MMAs
-// that read them complete, the V boxes (this slot's value columns) only after
-// P.V.  The next tiles' E boxes therefore load while a tile's softmax and P.V
-// run, and a V group has the MMAs of a whole tile to land in.  GLA and MLRA
-// have four stages and a one-box E group; their stage is one group, freed
-// after P.V.
+// bandwidth), the rest in shared memory.  TMEM columns: two score /
+// probability buffers of T, the output slice, the Q chunks.
 //
 // Warp roles (320 threads):
-//   warp 0     TMEM allocation; one thread streams the tiles (MLA: each tile's
-//              E group, then its V group) into a STAGES-deep ring with 2-D
-//              TMA loads (128-byte swizzle; a 128-token tile is two pages)
+//   warp 0     TMEM allocation; one thread streams the tiles into a
+//              STAGES-deep ring with 2-D TMA loads (128-byte swizzle; a
+//              128-token tile is two pages)
 //   warp 1     one thread issues S_j = Q K_j^T into one of two TMEM score
-//              buffers and P_{j-1} V_{j-1} into the TMEM output: for GLA and
-//              MLRA S_j, then P_{j-1} V_{j-1}; for MLA the E part of S_j,
-//              then the V part of S_j and P_{j-1} V_{j-1} in whichever order
-//              their inputs arrive.  The warp zeroes the rows of a tile past
-//              the context first (0 * NaN would poison the MMA)
+//              buffers, then P_{j-1} V_{j-1} into the TMEM output; the warp
+//              zeroes the rows of a tile past the context first (0 * NaN
+//              would poison the MMA)
 //   warps 2-9  two threads per head row, each owning half of the tile's
 //              columns and half of O's: read S_j from TMEM, exchange the tile
 //              maximum with the partner thread through shared memory, online
@@ -75,10 +60,8 @@ struct LatentSmem {
     unsigned char kv[STAGES][kStageBytes];
     float xmax[2][2][kRows];                  // [exchange parity][column half][row]
     uint32_t pvalid[kMaxSplitPages / 32];     // one bit per page of the part
-    uint64_t e_full[STAGES];                  // E group of the stage landed
-    uint64_t v_full[STAGES];                  // V group landed
-    uint64_t e_empty[STAGES];                 // score MMAs done with the E group
-    uint64_t v_empty[STAGES];                 // P.V done with the V group
+    uint64_t full[STAGES];                    // the stage's boxes landed
+    uint64_t empty[STAGES];                   // P.V done with the stage
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_ready;
@@ -106,27 +89,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
     pdl_launch_dependents();
-    const bool mla = !a.mlra && a.NU == 1;
     if (smem_u32(smem_raw) & 1023u) {
         // the 128-byte swizzle atoms need 1024-byte alignment; never expected
         if (threadIdx.x == 0)
             raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
         return;
     }
-    const int dn_boxes = a.dn / 64;
-    constexpr int NE = NKB - NVB;                                // E boxes: stage positions 0..NE-1
-    // Split release pays when the ring is shallow (MLA: two stages of nine
-    // boxes); with a deep ring and a one-box E group the whole stage is one
-    // group: loaded on e_full, freed by P.V on e_empty.
-    constexpr bool kSplit = NE > 1;
+    constexpr int NE = NKB - NVB;                                // rope boxes: stage positions 0..NE-1
+    static_assert(NE == 1, "one 64-wide rope key box");
     // Key box (64-column block of the slot's key row) at stage position p:
-    // E positions first (MLA: the other value half, then the rope key;
-    // GLA and MLRA: the rope key), the slot's value columns last.
-    auto key_box = [&](int p) -> int {
-        if (mla)
-            return p < NVB ? (slot ^ 1) * NVB + p : (p == NVB ? 2 * NVB : slot * NVB + (p - NE));
-        return p < NE ? NVB + p : p - NE;
-    };
+    // the rope key first, then the slot's latent (value) columns.
+    auto key_box = [&](int p) -> int { return p < NE ? NVB + p : p - NE; };
 
     int L = a.seq_lens[b];
     if (L > a.max_seq_len) {
@@ -141,10 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
-            mbar_init(&S.e_full[st], 1);
-            mbar_init(&S.v_full[st], 1);
-            mbar_init(&S.e_empty[st], 1);
-            mbar_init(&S.v_empty[st], 1);
+            mbar_init(&S.full[st], 1);
+            mbar_init(&S.empty[st], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
@@ -171,13 +142,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- TMA
         if (lane == 0 && n > 0) {
             prefetch_tmap(&kv_map);
-            const int unit_col0 = mla ? 0 : slot * a.dn;
+            const int unit_col0 = slot * a.dn;
             constexpr int kSubs = T >= kPage ? T / kPage : 1;   // pages a tile spans
             constexpr int kSubRows = T >= kPage ? kPage : T;    // rows per TMA box
-            int e_issued = 0, v_issued = 0;                     // tiles whose E / V group was started
-            // Start one group (positions [p_lo, p_hi)) of tile j on stage st;
-            // a tile with a bad page id loads nothing and only arrives.
-            auto load_group = [&](int j, int st, int p_lo, int p_hi, uint64_t *full) {
+            int issued = 0;                                     // tiles whose loads were started
+            for (; issued < n; ++issued) {
+                const int j = issued, st = j % STAGES;
+                if (j >= STAGES && !mbar_wait(&S.empty[st], ((j / STAGES) - 1) & 1)) {
+                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
+                    break;
+                }
+                // a tile with a bad page id loads nothing and only arrives
                 const int tok0 = p0 * kPage + j * T;
                 const int ntok = min(T, L - tok0);
                 const int nsub = (ntok + kSubRows - 1) / kSubRows;  // boxes of this tile holding context
@@ -190,68 +165,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                 }
                 if (!ok) {
-                    if (slot == 0 && p_lo == 0)
+                    if (slot == 0)
                         raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);
-                    mbar_arrive(full);
-                    return;
+                    mbar_arrive(&S.full[st]);
+                    continue;
                 }
-                mbar_arrive_expect_tx(full, (uint32_t)(nsub * (p_hi - p_lo) * kSubRows * 128));
+                mbar_arrive_expect_tx(&S.full[st], (uint32_t)(nsub * NKB * kSubRows * 128));
                 const int off = tok0 % kPage;
 #pragma unroll
                 for (int sub = 0; sub < kSubs; ++sub) {
                     if (sub >= nsub)
                         break;
                     const int y = (int)(pages[sub] * kPage) + off;
-                    for (int p = p_lo; p < p_hi; ++p) {
+                    for (int p = 0; p < NKB; ++p) {
                         const int kb = key_box(p);
-                        const int col = kb < dn_boxes ? unit_col0 + 64 * kb : a.NU * a.dn + 64 * (kb - dn_boxes);
-                        tma_load_2d(S.kv[st] + p * kBoxBytes + sub * kSubRows * 128, &kv_map, col, y, full);
+                        const int col = kb < NVB ? unit_col0 + 64 * kb : a.NU * a.dn + 64 * (kb - NVB);
+                        tma_load_2d(S.kv[st] + p * kBoxBytes + sub * kSubRows * 128, &kv_map, col, y, &S.full[st]);
                     }
-                }
-            };
-            if constexpr (!kSplit) {
-                for (; e_issued < n; ++e_issued) {
-                    const int j = e_issued, st = j % STAGES;
-                    if (j >= STAGES && !mbar_wait(&S.e_empty[st], ((j / STAGES) - 1) & 1)) {
-                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                        break;
-                    }
-                    load_group(j, st, 0, NKB, &S.e_full[st]);
-                }
-                v_issued = 0;
-            } else {
-                // E(j), then V(j): E(j+1) is not needed before V(j) has landed
-                // (S_{j+1} follows S_j), so the sequence costs nothing, and
-                // the thread sleeps in its waits instead of polling
-                for (int j = 0; j < n; ++j) {
-                    const int st = j % STAGES;
-                    const uint32_t eph = ((j / STAGES) - 1) & 1;
-                    if (j >= STAGES && !mbar_wait(&S.e_empty[st], eph)) {
-                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                        break;
-                    }
-                    load_group(j, st, 0, NE, &S.e_full[st]);
-                    e_issued = j + 1;
-                    if (j >= STAGES && !mbar_wait(&S.v_empty[st], eph)) {
-                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                        break;
-                    }
-                    load_group(j, st, NE, NKB, &S.v_full[st]);
-                    v_issued = j + 1;
                 }
             }
             // every copy this thread started has landed before the CTA can exit
-            for (int st = 0; st < STAGES; ++st) {
-                if (st < e_issued) {
-                    const int jl = st + ((e_issued - 1 - st) / STAGES) * STAGES;
-                    if (!mbar_wait(&S.e_full[st], (jl / STAGES) & 1))
-                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                }
-                if (st < v_issued) {
-                    const int jl = st + ((v_issued - 1 - st) / STAGES) * STAGES;
-                    if (!mbar_wait(&S.v_full[st], (jl / STAGES) & 1))
-                        raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
-                }
+            for (int st = 0; st < STAGES && st < issued; ++st) {
+                const int jl = st + ((issued - 1 - st) / STAGES) * STAGES;
+                if (!mbar_wait(&S.full[st], (jl / STAGES) & 1))
+                    raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
             }
         }
         __syncwarp();
@@ -260,22 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t qbase = smem_u32(&S.q[0][0]);
         bool ok = __all_sync(0xffffffffu, mbar_wait(&S.q_ready, 0));
         tc_fence_after();
-        // lane 0 (the issuing thread) tests a barrier; the warp follows its view
-        auto test = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return __shfl_sync(0xffffffffu, (lane == 0 && mbar_test(bar, parity)) ? 1 : 0, 0) != 0;
-        };
-        // zero rows [ntok, T) of stage positions [p_lo, p_hi) once the group's
-        // copies (whole boxes, rows past the context included) have landed;
-        // every lane observes the completed phase before it writes.  False
-        // (nothing written) if a lane's wait ran out.
-        auto zero_tail = [&](int st, int ntok, int p_lo, int p_hi, uint64_t *full, uint32_t parity) -> bool {
+        // zero rows [ntok, T) of stage st once its copies (whole boxes, rows
+        // past the context included) have landed; every lane observes the
+        // completed phase before it writes.  False (nothing written) if a
+        // lane's wait ran out.
+        auto zero_tail = [&](int st, int ntok, uint32_t parity) -> bool {
             if (ntok >= T)
                 return true;
-            if (!__all_sync(0xffffffffu, mbar_wait(full, parity)))
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.full[st], parity)))
                 return false;
-            const int rows = T - ntok, nb = p_hi - p_lo;
-            for (int idx = lane; idx < rows * nb * 8; idx += 32) {
-                const int box = p_lo + idx / (rows * 8), rem = idx % (rows * 8);
+            const int rows = T - ntok;
+            for (int idx = lane; idx < rows * NKB * 8; idx += 32) {
+                const int box = idx / (rows * 8), rem = idx % (rows * 8);
                 const int row = ntok + rem / 8, piece = rem % 8;
                 *reinterpret_cast<uint4 *>(S.kv[st] + box * kBoxBytes + row * 128 + piece * 16) =
                     make_uint4(0, 0, 0, 0);
@@ -293,13 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t kdesc0 = smem_desc(smem_u32(S.kv[0]), 16, 1024, 2);                      // K-major key boxes
         const uint64_t vdesc0 = smem_desc(smem_u32(S.kv[0]) + NE * kBoxBytes, kBoxBytes, 1024, 2);  // MN-major values
         const uint64_t qdesc0 = smem_desc(qbase, 16, 1024, 2);
-        // score MMAs of stage positions [PLO, PHI) of tile j
-        auto issue_s = [&](int j, auto PLO, auto PHI) {
+        // the score MMAs of tile j
+        auto issue_s = [&](int j) {
             if (lane == 0) {
                 const uint32_t d = tS + (j & 1) * T;
                 const uint64_t kd = kdesc0 + (uint64_t)((j % STAGES) * kStageUnits);
 #pragma unroll
-                for (int p = decltype(PLO)::value; p < decltype(PHI)::value; ++p) {
+                for (int p = 0; p < NKB; ++p) {
                     const int kb = key_box(p);
                     if (kb < NQT) {
                         const uint32_t qa = tQ + kb * 32;
@@ -316,10 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        using P0 = std::integral_constant<int, 0>;
-        using PE = std::integral_constant<int, NE>;
-        using PK = std::integral_constant<int, NKB>;
-        // P_t V_t into O (P_t is ready); frees tile t's V group
+        // P_t V_t into O (P_t is ready); frees tile t's stage
         auto issue_pv = [&](int t) {
             tc_fence_after();
             if (lane == 0) {
@@ -329,92 +259,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int k = 0; k < T / 16; ++k)
                     umma_ts(tO, pa + 8 * k, vd + (uint64_t)(k * 128), kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
                 umma_commit(&S.o_ready);
-                umma_commit(kSplit ? &S.v_empty[t % STAGES] : &S.e_empty[t % STAGES]);
+                umma_commit(&S.empty[t % STAGES]);
             }
             __syncwarp();
         };
-        if constexpr (!kSplit) {
-            // S_j as soon as its stage is in, then P_{j-1} V_{j-1}
-            for (int j = 0; ok && j < n; ++j) {
-                const int st = j % STAGES;
-                const uint32_t fph = (j / STAGES) & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&S.e_full[st], fph))) {
-                    ok = false;
-                    break;
-                }
-                if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, j), 0, NKB, &S.e_full[st], fph)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                issue_s(j, P0{}, PK{});
-                if (lane == 0)
-                    umma_commit(&S.s_full[j & 1]);
-                __syncwarp();
-                if (j >= 1) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(&S.p_full[(j - 1) & 1], ((j - 1) >> 1) & 1)))
-                        ok = false;
-                    else
-                        issue_pv(j - 1);
-                }
+        // S_j as soon as its stage is in, then P_{j-1} V_{j-1}
+        for (int j = 0; ok && j < n; ++j) {
+            const int st = j % STAGES;
+            const uint32_t fph = (j / STAGES) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.full[st], fph))) {
+                ok = false;
+                break;
             }
-            if (ok && n > 0) {
-                if (__all_sync(0xffffffffu, mbar_wait(&S.p_full[(n - 1) & 1], ((n - 1) >> 1) & 1)))
-                    issue_pv(n - 1);
+            if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, j), fph)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            issue_s(j);
+            if (lane == 0)
+                umma_commit(&S.s_full[j & 1]);
+            __syncwarp();
+            if (j >= 1) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&S.p_full[(j - 1) & 1], ((j - 1) >> 1) & 1)))
+                    ok = false;
                 else
-                    ok = false;
+                    issue_pv(j - 1);
             }
-        } else {
-            // Three kinds of work, issued as their inputs arrive (the V part of
-            // the open score tile first, so its softmax starts early, then P.V,
-            // then the next tile's E part):
-            //   PV_t     needs P_t (so S_t is complete)
-            //   S_t(V)   needs the V group of tile t and S_t(E)
-            //   S_t(E)   needs the E group of tile t, S_{t-1}(V) (scores complete in
-            //            tile order) and PV_{t-2} (S_t reuses the buffer P_{t-2} was in;
-            //            MMAs run in issue order)
-            int jpv = 0, jsv = 0, jse = 0;             // next tile of each kind
-            uint32_t idle = 0;
-            while (ok && jpv < n) {
-                if (jsv < jse && test(&S.v_full[jsv % STAGES], (jsv / STAGES) & 1)) {
-                    const int st = jsv % STAGES;
-                    if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jsv), NE, NKB, &S.v_full[st], (jsv / STAGES) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_s(jsv, PE{}, PK{});
-                    if (lane == 0)
-                        umma_commit(&S.s_full[jsv & 1]);
-                    __syncwarp();
-                    ++jsv;
-                    idle = 0;
-                    continue;
-                }
-                if (jpv < jsv && test(&S.p_full[jpv & 1], (jpv >> 1) & 1)) {
-                    issue_pv(jpv);
-                    ++jpv;
-                    idle = 0;
-                    continue;
-                }
-                if (jse < n && jse == jsv && jpv >= jse - 1 && test(&S.e_full[jse % STAGES], (jse / STAGES) & 1)) {
-                    const int st = jse % STAGES;
-                    if (!zero_tail(st, tile_ntok<T>(S.pvalid, L, p0, jse), 0, NE, &S.e_full[st], (jse / STAGES) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_s(jse, P0{}, PE{});
-                    if (lane == 0)
-                        umma_commit(&S.e_empty[st]);
-                    __syncwarp();
-                    ++jse;
-                    idle = 0;
-                    continue;
-                }
-                if (++idle >= kWaitLimit)
-                    ok = false;
-            }
+        }
+        if (ok && n > 0) {
+            if (__all_sync(0xffffffffu, mbar_wait(&S.p_full[(n - 1) & 1], ((n - 1) >> 1) & 1)))
+                issue_pv(n - 1);
+            else
+                ok = false;
         }
         if (!ok && lane == 0)
             raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
@@ -434,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = sw >> 2;                                // column half
         const int h = quarter * 32 + lane;                       // head row = TMEM lane
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const int rows_used = a.mlra || mla ? a.H : a.HPU;      // GLA: the group's heads
+        const int rows_used = a.mlra ? a.H : a.HPU;             // GLA: the group's heads
         {
             // validity of every page of this part (read by the MMA warp and here)
             const int npg = min(a.pages_per_split, max(0, (L + kPage - 1) / kPage - p0));
@@ -452,8 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 size_t row;
                 if (a.mlra)
                     row = ((size_t)b * a.H + h) * a.NU + slot;
-                else if (mla)
-                    row = (size_t)b * a.H + h;
                 else
                     row = (size_t)b * a.H + (size_t)slot * a.HPU + h;
                 qn = a.q_nope + row * a.dn;
@@ -463,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = half; kb < NKB; kb += 2) {
                 const __nv_bfloat16 *src = nullptr;
                 if (qn)
-                    src = kb < dn_boxes ? qn + 64 * kb : qr + 64 * (kb - dn_boxes);
+                    src = kb < NVB ? qn + 64 * kb : qr + 64 * (kb - NVB);
                 if (kb < NQT) {
                     uint32_t r[32];
 #pragma unroll
@@ -622,37 +497,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
         }
         const bool valid = h < rows_used;
-        int hu, col0;
-        if (a.mlra) {
-            hu = h * a.NU + slot;
-            col0 = 0;
-        } else if (mla) {
-            hu = h;
-            col0 = slot * kDvSlot;
-        } else {
-            hu = slot * a.HPU + h;
-            col0 = 0;
-        }
+        const int hu = a.mlra ? h * a.NU + slot : slot * a.HPU + h;
         const size_t prow = ((size_t)b * a.num_splits + split) * a.HU + (valid ? hu : 0);
-        float *dst = a.po + prow * a.dn + col0 + half * OH;
+        float *dst = a.po + prow * a.dn + half * OH;
         const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-        uint32_t r[64];
+        constexpr int CH = OH < 64 ? OH : 64;                     // columns per TMEM load
+        uint32_t r[CH];
 #pragma unroll 1
-        for (int c = 0; c < OH / 64; ++c) {
-            if (have)
-                tmem_ld64(tO + lane_addr + half * OH + 64 * c, r);
+        for (int c = 0; c < OH / CH; ++c) {
+            if (have) {
+                if constexpr (CH == 64)
+                    tmem_ld64(tO + lane_addr + half * OH + CH * c, r);
+                else
+                    tmem_ld32(tO + lane_addr + half * OH + CH * c, r);
+            }
             if (valid) {
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
+                for (int i = 0; i < CH; i += 4) {
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (have)
                         v = make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
                                         __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
-                    *reinterpret_cast<float4 *>(dst + 64 * c + i) = v;
+                    *reinterpret_cast<float4 *>(dst + CH * c + i) = v;
                 }
             }
         }
-        if (valid && half == 0 && (!mla || slot == 0))
+        if (valid && half == 0)
             a.plse[prow] = (have && l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
     }
     __syncwarp();
@@ -685,31 +555,31 @@ cudaError_t launch_latent(const DecodeArgs &a, int slots, cudaStream_t st)
 
 }  // namespace
 
-// Shapes the tensor-core latent kernel covers: MLA 512 + 64 (two value
-// halves), GLA with 256-wide latent heads + 64 rope, MLRA with 128-wide
-// branches + 64 rope; at most 128 query heads per MMA.
-// Pages per part must be a whole number of tiles and fit the validity table.
-int latent_tc_page_multiple(const Problem &pr) { return pr.mlra ? 2 : 1; }
+// Shapes the tensor-core latent kernel covers: GLA or MLRA (any number of
+// groups or branches, one of them included) with latent slices of 64, 128 or
+// 256 columns and a 64-wide rope key; at most 128 query heads per MMA.  Pages
+// per part must be a whole number of tiles and fit the validity table.
+int latent_tc_page_multiple(const Problem &pr) { return pr.dn <= 128 ? 2 : 1; }
 int latent_tc_max_pages_per_split() { return kMaxSplitPages; }
 
 int latent_tc_slots(const Problem &pr)
 {
-    if (!pr.latent || pr.dr != 64)
+    if (!pr.latent || pr.dr != 64 || (pr.variant != KVATTN_GLA && !pr.mlra))
         return 0;
-    if (pr.mlra)
-        return (pr.dn == 128 && pr.H <= kRows) ? pr.NU : 0;
-    if (pr.NU == 1)
-        return (pr.dn == 512 && pr.H <= kRows) ? 2 : 0;
-    return (pr.dn == 256 && pr.HPU <= kRows) ? pr.NU : 0;
+    if (pr.dn != 64 && pr.dn != 128 && pr.dn != 256)
+        return 0;
+    return (pr.mlra ? pr.H : pr.HPU) <= kRows ? pr.NU : 0;
 }
 
 cudaError_t launch_latent_tc(const DecodeArgs &a, const Problem &pr, cudaStream_t st)
 {
     const int slots = latent_tc_slots(pr);
-    if (pr.mlra)
+    // <tokens per tile, key boxes, value boxes, stages, Q chunks in TMEM>;
+    // TMEM columns 2 T + 64 value boxes + 32 Q chunks stay within 512
+    if (pr.dn == 64)
+        return launch_latent<128, 2, 1, 4, 2>(a, slots, st);
+    if (pr.dn == 128)
         return launch_latent<128, 3, 2, 4, 3>(a, slots, st);
-    if (pr.NU == 1)
-        return launch_latent<64, 9, 4, 2, 4>(a, slots, st);
     return launch_latent<64, 5, 4, 4, 4>(a, slots, st);
 }
 

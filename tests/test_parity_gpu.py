@@ -73,6 +73,14 @@ SMALL = {
     "mlra": (W.WORKLOADS["mlra_128k"].replace(batch=2, ctx=(100, 700)), None),
     "gqa_contiguous": (W.WORKLOADS["gqa"].replace(batch=2, ctx=(1, 300), paged=False), None),
     "mlra_fp32_out": (W.WORKLOADS["mlra_128k"].replace(batch=1, ctx=(333, 333), out_dtype="fp32"), None),
+    # more groups / branches on the same tensor-core kernel, and the single
+    # group or branch a tensor-parallel rank holds
+    "gla1_shard": (W.WORKLOADS["gla"].replace(batch=2, num_q_heads=64, num_kv=1, ctx=(100, 700)), None),
+    "gla4": (W.WORKLOADS["gla"].replace(batch=2, num_kv=4, d_nope=128, ctx=(100, 700)), None),
+    "gla8": (W.WORKLOADS["gla"].replace(batch=2, num_kv=8, d_nope=64, ctx=(100, 700)), None),
+    "mlra1_shard": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=1, ctx=(100, 700)), None),
+    "mlra2": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=2, d_nope=256, ctx=(100, 700)), None),
+    "mlra8": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=8, d_nope=64, ctx=(100, 700)), None),
 }
 
 
@@ -148,6 +156,8 @@ def test_benchmark_shapes_use_the_specialised_kernels(dev):
     for n in ("gla", "mlra_128k", "mlra_1m", "mlra_b8_128k"):
         assert kernel_of(W.WORKLOADS[n]) == "latent_tc", n
     assert kernel_of(W.WORKLOADS["tiny_mla"]) == "generic"
+    for name in ("gla1_shard", "gla4", "gla8", "mlra1_shard", "mlra2", "mlra8"):
+        assert kernel_of(SMALL[name][0]) == "latent_tc", name
 
 
 def test_tiny_config_exact_shape(dev, oracle_mod):
@@ -299,3 +309,17 @@ def test_gqa_plan_merges_in_kernel(dev):
         plan = K.kvattn_get_plan(s.variant_id, K.params_for(s, (hi + 63) // 64, 1 << 20, hi))
         assert plan.launches == launches, name
         assert plan.header_bytes >= 256
+
+
+@pytest.mark.parametrize("name,world", [("mlra_128k", 4), ("mlra_128k", 2), ("gla", 2)])
+def test_tensor_parallel_shards_on_one_device(dev, oracle_mod, name, world):
+    """What each tensor-parallel rank computes (its MLRA branches or GLA
+    groups, through the library), solved in turn on one GPU and assembled as
+    the collective would (branch outputs summed in fp32, heads side by side),
+    against the oracle on the whole problem."""
+    from shared_kv_caches_b200 import tp as TP
+    shape = W.WORKLOADS[name].replace(batch=2, ctx=(300, 900))
+    x = W.make_inputs(shape, seed=12)
+    out, lse = TP.tp_decode_one_device(x, world, dev)
+    ref_out, ref_lse = oracle_mod.decode(x)
+    check(out, lse, ref_out, ref_lse, what=f"tp {name} x{world}")
