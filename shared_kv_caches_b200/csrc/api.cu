@@ -150,10 +150,10 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
         pl->head_chunk = 32;
         pl->head_chunks = 1;
         base = (long long)pr.B * pr.NU;
-        // about 2.5 waves of one CTA per SM: measured on 32 x U[1024,8192]
-        // contexts, 12 parts decode as fast as 18 and leave the combine a
-        // third less to merge (65.8 against 67.5 us per step); 8 parts is slower
-        splits = choose_splits(forced_splits, base, max_pages, 5LL * num_sms / 2, 2);
+        // about 1.3 waves of one CTA per SM: measured on 32 x U[1024,8192]
+        // contexts (decode + combine), 6 parts 48.3 us, 7 parts 49.8, 12 parts
+        // 54.3, 8 parts 60.1 (1.7 waves), 4 parts 60.4 (under one wave)
+        splits = choose_splits(forced_splits, base, max_pages, 13LL * num_sms / 10, 2);
     } else {
         const int hc = generic_head_chunk(pr);
         if (!hc)

@@ -79,7 +79,7 @@ def test_plan_every_workload(lib, name):
 EXPECTED_PLANS = {
     "gla": ("latent_tc", 4, 64, 512, 2),
     "gqa": ("gqa", 7, 19, 1792, 1),
-    "mfa": ("mqa_tc", 12, 11, 384, 2),
+    "mfa": ("mqa_tc", 6, 22, 192, 2),
     "mla": ("latent_pair", 5, 103, 640, 2),
     "mlra_128k": ("latent_tc", 37, 56, 148, 2),
     "mlra_512k": ("latent_tc", 37, 222, 148, 2),
