@@ -29,8 +29,8 @@
  *               the R normalised branch outputs are summed (latent space)
  *
  * Memory (all device pointers, row-major, caller-owned):
- *   q_nope     bf16 [B][H][d_nope]           (MLRA [B][H][R][d_nope])
- *   q_rope     bf16 [B][H][d_rope]           (MLRA [B][H][R][d_rope]); NULL when
+ *   q_nope     bf16 [B][Q][H][d_nope]        (MLRA [B][Q][H][R][d_nope]), Q = q_len
+ *   q_rope     bf16 [B][Q][H][d_rope]        (MLRA [B][Q][H][R][d_rope]); NULL when
  *              d_rope == 0 (GQA/MQA)
  *   kv_cache   latent variants: bf16 [num_pages][page_size][num_kv*d_nope + d_rope],
  *              each token row [c_0 | ... | c_{num_kv-1} | k_rope];
@@ -39,8 +39,8 @@
  *              64-token page; NULL = contiguous cache, sequence b owns pages
  *              b*max_pages_per_seq .. b*max_pages_per_seq + max_pages_per_seq-1
  *   seq_lens   int32 [B], 0 <= seq_lens[b] <= max_seq_len (read on the device)
- *   out        [B][H][d_nope], bf16 (round to nearest even) or fp32
- *   lse        fp32 [B][H] (MLRA [B][H][R]), natural log of the softmax
+ *   out        [B][Q][H][d_nope], bf16 (round to nearest even) or fp32
+ *   lse        fp32 [B][Q][H] (MLRA [B][Q][H][R]), natural log of the softmax
  *              denominator including sm_scale; may be NULL
  *   workspace  device scratch of kvattn_workspace_size() bytes, 256-byte
  *              aligned, prepared once with kvattn_workspace_init()
@@ -48,6 +48,13 @@
  * Token j of sequence b is slot j % 64 of page block_table[b][j / 64].
  * Slots past seq_lens[b] may hold anything (NaN included) and never reach a
  * result.  An empty sequence yields out = 0 and lse = -inf.
+ *
+ * Several query tokens per sequence (q_len = Q > 1: speculative or
+ * multi-token-prediction decode; the GLA page contrasts query length 1 with
+ * longer queries): the Q newest tokens of each sequence are already in the
+ * cache (seq_lens counts them), and query position i (0-based) attends the
+ * cache up to and including its own token, seq_lens[b] - (Q - 1 - i) tokens
+ * (causal).  Each position reads its prefix of the cache on its own.
  *
  * Conventions: every call is asynchronous on `stream` (a cudaStream_t, NULL =
  * legacy default stream) and returns a status before or after enqueueing;
@@ -128,6 +135,8 @@ typedef struct {
     int32_t max_seq_len;       /* >= every seq_lens[b]; <= capacity */
     int32_t num_splits;        /* 0 = library choice, > 0 forces */
     int32_t out_dtype;         /* kvattn_out_dtype */
+    int32_t q_len;             /* query tokens per sequence, 1..64 (0 means 1); batch * q_len
+                                  <= 65535 */
 } kvattn_params;
 
 /* What kvattn_decode will launch for a problem (see kvattn_get_plan). */
@@ -262,7 +271,7 @@ int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code);
 /* Static, human-readable name of a status code. */
 const char *kvattn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 200 (kvattn_params carries q_len). */
 int kvattn_version(void);
 
 #ifdef __cplusplus

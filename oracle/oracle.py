@@ -106,14 +106,56 @@ def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None
 
     Returns ``(out, lse)``: out ``[n_b][n_h][d_nope]`` float64 (MLRA: the sum
     over branches), lse ``[n_b][n_h]`` (MLRA ``[n_b][n_h][R]``), natural log.
-    ``b_list`` / ``h_list`` select sequences / heads (default: all).
+    ``b_list`` / ``h_list`` select sequences / heads (default: all).  With
+    several query tokens per sequence (``shape.q_len`` = Q > 1) the results
+    carry a query axis after the sequence axis: see ``decode_queries``.
     """
     s = inputs["shape"]
+    if getattr(s, "q_len", 1) > 1:
+        return decode_queries(inputs, b_list, nthreads, sm_scale, h_list)
     scale = inputs["sm_scale"] if sm_scale is None else sm_scale
     return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
                 inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 0,
                 inputs["q_nope"], inputs["q_rope"], inputs["kv"], inputs["block_table"],
                 inputs["seq_lens"], scale, b_list, nthreads, h_list)
+
+
+def decode_queries(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None):
+    """Decode with Q > 1 query tokens per sequence (speculative or multi-token
+    decode; the GLA page sets query length 1 against longer queries).
+
+    The Q newest tokens of sequence b are already in its cache (seq_lens[b]
+    counts them); query position i attends the cache up to and including its
+    own token, the first seq_lens[b] - (Q - 1 - i) tokens (causal masking
+    among the new tokens).  Each (sequence, position) is therefore a
+    single-token decode over that prefix of the same pages, which is how this
+    computes it.  Returns out ``[n_b][Q][n_h][d_nope]`` and lse
+    ``[n_b][Q][n_h]`` (MLRA ``[n_b][Q][n_h][R]``).
+    """
+    s = inputs["shape"]
+    Q = s.q_len
+    B = s.batch
+    bs = np.arange(B) if b_list is None else np.asarray(b_list)
+    lens = np.asarray(inputs["seq_lens"], dtype=np.int64)
+    # one row per (sequence, position): its own query, the sequence's pages,
+    # the causal prefix length
+    q_nope = np.asarray(inputs["q_nope"])
+    q_rope = None if inputs["q_rope"] is None else np.asarray(inputs["q_rope"])
+    rows_q = q_nope.reshape((B * Q,) + q_nope.shape[2:])
+    rows_qr = None if q_rope is None else q_rope.reshape((B * Q,) + q_rope.shape[2:])
+    rows_len = np.maximum(np.repeat(lens, Q) - np.tile(Q - 1 - np.arange(Q), B), 0).astype(np.int32)
+    bt = inputs["block_table"]
+    if bt is None:
+        # contiguous: sequence b owns pages b*mpps .. ; row v keeps its sequence's pages
+        mpps = inputs["max_pages_per_seq"]
+        rows_bt = np.repeat(np.arange(B, dtype=np.int32)[:, None] * mpps + np.arange(mpps, dtype=np.int32), Q, axis=0)
+    else:
+        rows_bt = np.repeat(np.asarray(bt), Q, axis=0)
+    rows = dict(inputs, shape=s.replace(batch=B * Q, q_len=1, paged=True), q_nope=rows_q, q_rope=rows_qr,
+                seq_lens=rows_len, block_table=np.ascontiguousarray(rows_bt, dtype=np.int32))
+    sel = (bs[:, None] * Q + np.arange(Q)).reshape(-1)
+    out, lse = decode(rows, b_list=sel, nthreads=nthreads, sm_scale=sm_scale, h_list=h_list)
+    return out.reshape((len(bs), Q) + out.shape[1:]), lse.reshape((len(bs), Q) + lse.shape[1:])
 
 
 def decode_f64(variant, num_kv, q_nope, q_rope, kv, seq_lens, sm_scale, block_table=None,

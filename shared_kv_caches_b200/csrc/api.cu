@@ -27,7 +27,10 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
         return KVATTN_ERR_INVALID_ARG;
     if (p->out_dtype != KVATTN_OUT_BF16 && p->out_dtype != KVATTN_OUT_FP32)
         return KVATTN_ERR_INVALID_ARG;
-    if (p->batch > 65535 || p->num_q_heads > 65535)
+    if (p->q_len < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    const int q_len = p->q_len > 0 ? p->q_len : 1;
+    if (q_len > kMaxQueryLen || (long long)p->batch * q_len > 65535 || p->num_q_heads > 65535)
         return KVATTN_ERR_UNSUPPORTED;
     if (p->page_size != kPage)
         return KVATTN_ERR_UNSUPPORTED;
@@ -52,7 +55,8 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
         return KVATTN_ERR_UNSUPPORTED;
 
     pr->variant = variant;
-    pr->B = p->batch;
+    pr->B = p->batch * q_len;     // one row per (sequence, query position)
+    pr->q_len = q_len;
     pr->H = p->num_q_heads;
     pr->NU = p->num_kv;
     pr->dn = p->d_nope;
@@ -239,7 +243,7 @@ int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, c
 
 using namespace kvattn;
 
-extern "C" int kvattn_version(void) { return 100; }
+extern "C" int kvattn_version(void) { return 200; }
 
 extern "C" const char *kvattn_status_string(int status)
 {
@@ -326,6 +330,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     a.lse_out = lse;
     a.out_fp32 = pr.out_dtype == KVATTN_OUT_FP32;
     a.B = pr.B;
+    a.q_len = pr.q_len;
     a.H = pr.H;
     a.NU = pr.NU;
     a.dn = pr.dn;

@@ -55,14 +55,7 @@ __global__ void __launch_bounds__(kThreads) generic_decode_kernel(const DecodeAr
     uint32_t *ks = reinterpret_cast<uint32_t *>(smem + ((HC * Dk + HC * kPage + 3 * HC) * 4 + 15) / 16 * 16);
     uint32_t *vs = ks + kPage * KS / 2;                    // GQA/MQA value rows
 
-    int L = a.seq_lens[b];
-    if (L > a.max_seq_len) {
-        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
-        L = a.max_seq_len;
-    }
-    if (L < 0)
-        L = 0;
+    const int L = row_context(a, b, tid == 0 && blockIdx.x == 0 && blockIdx.y == 0);
     const int npages = (L + kPage - 1) / kPage;
     const int p0 = s * a.pages_per_split;
     const int p1 = min(npages, p0 + a.pages_per_split);
@@ -98,8 +91,7 @@ __global__ void __launch_bounds__(kThreads) generic_decode_kernel(const DecodeAr
     const int vec_k = Dk / 8;     // 16-byte vectors per key row
     const int vec_v = Dv / 8;
     for (int pi = p0; pi < p1; ++pi) {
-        const long long page = a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi]
-                                             : (long long)b * a.mpps + pi;
+        const long long page = row_page(a, b, pi);
         if (page < 0 || page >= a.num_pages) {
             if (tid == 0)
                 raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);

@@ -101,13 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the rope key first, then the slot's latent (value) columns.
     auto key_box = [&](int p) -> int { return p < NE ? NVB + p : p - NE; };
 
-    int L = a.seq_lens[b];
-    if (L > a.max_seq_len) {
-        if (threadIdx.x == 0 && split == 0 && slot == 0)
-            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
-        L = a.max_seq_len;
-    }
-    L = max(L, 0);
+    const int L = row_context(a, b, threadIdx.x == 0 && split == 0 && slot == 0);
     const int p0 = split * a.pages_per_split;
     const int tok_end = min(L, (p0 + a.pages_per_split) * kPage);
     const int n = tok_end > p0 * kPage ? (tok_end - p0 * kPage + T - 1) / T : 0;

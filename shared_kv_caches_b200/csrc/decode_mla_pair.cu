@@ -126,13 +126,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kThreads, 1)
         return;
     }
 
-    int L = a.seq_lens[b];
-    if (L > a.max_seq_len) {
-        if (threadIdx.x == 0 && split == 0 && r == 0)
-            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
-        L = a.max_seq_len;
-    }
-    L = max(L, 0);
+    const int L = row_context(a, b, threadIdx.x == 0 && split == 0 && r == 0);
     const int p0 = split * a.pages_per_split;
     const int tok_end = min(L, (p0 + a.pages_per_split) * kPage);
     const int n = tok_end > p0 * kPage ? (tok_end - p0 * kPage + kPage - 1) / kPage : 0;   // pages

@@ -89,13 +89,7 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     pdl_launch_dependents();
 
-    int L = a.seq_lens[b];
-    if (L > a.max_seq_len) {
-        if (threadIdx.x == 0 && split == 0 && kvh == 0)
-            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
-        L = a.max_seq_len;
-    }
-    L = max(L, 0);
+    const int L = row_context(a, b, threadIdx.x == 0 && split == 0 && kvh == 0);
     const int npages = (L + kPage - 1) / kPage;
     const int p0 = split * a.pages_per_split;
     const int n = max(0, min(npages, p0 + a.pages_per_split) - p0);
@@ -119,8 +113,7 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
                     break;
                 }
                 const int pi = p0 + i;
-                const long long page = a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi]
-                                                     : (long long)b * a.mpps + pi;
+                const long long page = row_page(a, b, pi);
                 if (page < 0 || page >= a.num_pages) {
                     raise_error(a.err, KVATTN_DEVERR_PAGE_OUT_OF_RANGE);
                     S.skip[st] = 1;

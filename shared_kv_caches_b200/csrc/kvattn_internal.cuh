@@ -15,11 +15,13 @@ constexpr int kPage = 64;               // tokens per cache page
 constexpr int kDefaultSMs = 148;        // B200; used when no device can be queried
 constexpr size_t kWsHeader = 256;       // workspace header: device error word
 constexpr int kMaxSplits = 1024;
+constexpr int kMaxQueryLen = 64;        // query tokens per sequence in one call
 
 // Validated problem, host side.
 struct Problem {
     int variant;
-    int B, H, NU, dn, dr;
+    int B, H, NU, dn, dr;  // B: rows = sequences x query tokens
+    int q_len;         // query tokens per sequence
     int Dk, Dv;        // key width (d_nope + d_rope) and value width (d_nope)
     int row;           // elements per token row of a page (per K or V plane for GQA/MQA)
     int HPU;           // query heads served by one unit (KV head / group / branch)
@@ -47,6 +49,7 @@ struct DecodeArgs {
     int mpps, num_pages, max_seq_len;
     int num_splits, pages_per_split, head_chunks;
     int latent, mlra;
+    int q_len;                    // query tokens per sequence; B counts (sequence, position) rows
     float scale_log2;             // sm_scale * log2(e): scores kept in base 2
 };
 
@@ -59,6 +62,30 @@ struct CombineArgs {
 };
 
 __device__ __forceinline__ void raise_error(int *err, int bit) { atomicOr(err, bit); }
+
+// Row v of a decode call is query position v % q_len of sequence v / q_len.
+// Position i of the q_len newest tokens attends the cache up to and
+// including itself: seq_lens[s] - (q_len - 1 - i) tokens (causal).  A
+// sequence longer than max_seq_len sets the error bit (in the first CTA of
+// its rows that reads it) and is clamped.
+__device__ __forceinline__ int row_context(const DecodeArgs &a, int v, bool report)
+{
+    const int s = v / a.q_len, pos = v % a.q_len;
+    int L = a.seq_lens[s];
+    if (L > a.max_seq_len) {
+        if (report)
+            raise_error(a.err, KVATTN_DEVERR_SEQ_TOO_LONG);
+        L = a.max_seq_len;
+    }
+    return max(L - (a.q_len - 1 - pos), 0);
+}
+
+// Physical page of logical page pi of row v's sequence.
+__device__ __forceinline__ long long row_page(const DecodeArgs &a, int v, int pi)
+{
+    const long long s = v / a.q_len;
+    return a.block_table ? (long long)a.block_table[s * a.mpps + pi] : s * a.mpps + pi;
+}
 
 // Programmatic dependent launch: a decode kernel lets the combine pass queued
 // behind it be scheduled at once (its blocks then wait in pdl_wait_primary

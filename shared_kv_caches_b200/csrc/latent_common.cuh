@@ -78,10 +78,7 @@ __device__ __forceinline__ float reduce_extreme(const float *v)
     return kMax ? fmax3(x, y, z) : fmin3(x, y, z);
 }
 
-__device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi)
-{
-    return a.block_table ? (long long)a.block_table[(size_t)b * a.mpps + pi] : (long long)b * a.mpps + pi;
-}
+__device__ __forceinline__ long long page_id(const DecodeArgs &a, int b, int pi) { return row_page(a, b, pi); }
 
 __device__ __forceinline__ bool page_ok(const DecodeArgs &a, long long page)
 {

@@ -43,7 +43,7 @@ KVATTN_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 class kvattn_params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "num_q_heads", "num_kv", "d_nope", "d_rope", "page_size", "max_pages_per_seq",
-        "num_pages", "max_seq_len", "num_splits", "out_dtype")]
+        "num_pages", "max_seq_len", "num_splits", "out_dtype", "q_len")]
 
 
 class kvattn_plan(ctypes.Structure):
@@ -94,10 +94,10 @@ def load():
 
 
 def make_params(batch, num_q_heads, num_kv, d_nope, d_rope, max_pages_per_seq, num_pages,
-                max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64) -> kvattn_params:
+                max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64, q_len=1) -> kvattn_params:
     return kvattn_params(int(batch), int(num_q_heads), int(num_kv), int(d_nope), int(d_rope),
                          int(page_size), int(max_pages_per_seq), int(num_pages), int(max_seq_len),
-                         int(num_splits), int(out_dtype))
+                         int(num_splits), int(out_dtype), int(q_len))
 
 
 def kvattn_version() -> int:
@@ -178,7 +178,7 @@ def params_for(shape, max_pages_per_seq, num_pages, max_seq_len, num_splits=0) -
     return make_params(shape.batch, shape.num_q_heads, shape.num_kv, shape.d_nope, shape.d_rope,
                        max_pages_per_seq, num_pages, max_seq_len, num_splits,
                        KVATTN_OUT_FP32 if shape.out_dtype == "fp32" else KVATTN_OUT_BF16,
-                       shape.page_size)
+                       shape.page_size, shape.q_len)
 
 
 def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, sm_scale, out, lse,

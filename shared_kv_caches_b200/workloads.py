@@ -70,6 +70,7 @@ class Shape:
     out_dtype: str = "bf16"
     sm_scale: float | None = None
     input_scale: float = 1.0
+    q_len: int = 1          # query tokens per sequence (the newest q_len cached tokens)
 
     @property
     def variant_id(self) -> int:
@@ -113,25 +114,29 @@ class Shape:
             return float(self.sm_scale)
         return 1.0 / math.sqrt(self.key_dim)
 
+    def _rows(self) -> tuple:
+        """Leading axes: sequence, and query token when there are several."""
+        return (self.batch,) if self.q_len == 1 else (self.batch, self.q_len)
+
     def q_nope_shape(self) -> tuple:
         if self.variant == "mlra":
-            return (self.batch, self.num_q_heads, self.num_kv, self.d_nope)
-        return (self.batch, self.num_q_heads, self.d_nope)
+            return self._rows() + (self.num_q_heads, self.num_kv, self.d_nope)
+        return self._rows() + (self.num_q_heads, self.d_nope)
 
     def q_rope_shape(self) -> tuple | None:
         if self.d_rope == 0:
             return None
         if self.variant == "mlra":
-            return (self.batch, self.num_q_heads, self.num_kv, self.d_rope)
-        return (self.batch, self.num_q_heads, self.d_rope)
+            return self._rows() + (self.num_q_heads, self.num_kv, self.d_rope)
+        return self._rows() + (self.num_q_heads, self.d_rope)
 
     def out_shape(self) -> tuple:
-        return (self.batch, self.num_q_heads, self.d_nope)
+        return self._rows() + (self.num_q_heads, self.d_nope)
 
     def lse_shape(self) -> tuple:
         if self.variant == "mlra":
-            return (self.batch, self.num_q_heads, self.num_kv)
-        return (self.batch, self.num_q_heads)
+            return self._rows() + (self.num_q_heads, self.num_kv)
+        return self._rows() + (self.num_q_heads,)
 
     def pool_shape(self, num_pages: int) -> tuple:
         if self.latent:

@@ -419,3 +419,69 @@ def test_sample_of_sequences_matches_full(oracle_mod):
     o4, l4 = oracle_mod.decode(y, b_list=[1], h_list=[3])
     np.testing.assert_array_equal(o4[0, 0], out[1, 3])
     np.testing.assert_array_equal(l4[0, 0], lse[1, 3])
+
+
+# ----------------------------------------------------- several query tokens
+
+def _q_shape(name, q_len):
+    base = {"mla": W.WORKLOADS["mla"].replace(num_q_heads=4, d_nope=64, d_rope=16),
+            "mlra": W.WORKLOADS["mlra_128k"].replace(num_q_heads=4, num_kv=2, d_nope=32, d_rope=16),
+            "gqa": W.WORKLOADS["gqa"].replace(num_q_heads=4, num_kv=2, d_nope=32)}[name]
+    return base.replace(batch=2, ctx=(20, 150), q_len=q_len)
+
+
+@pytest.mark.parametrize("name", ["mla", "mlra", "gqa"])
+def test_queries_last_position_sees_the_whole_context(oracle_mod, name):
+    """The newest query token attends every cached token: it equals the
+    single-token decode of that token's query."""
+    x = W.make_inputs(_q_shape(name, 3), seed=21)
+    out, lse = oracle_mod.decode(x)
+    single = dict(x, shape=x["shape"].replace(q_len=1), q_nope=x["q_nope"][:, -1],
+                  q_rope=None if x["q_rope"] is None else x["q_rope"][:, -1])
+    ref_out, ref_lse = oracle_mod.decode(single)
+    np.testing.assert_allclose(out[:, -1], ref_out, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, -1], ref_lse, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("name", ["mla", "gqa"])
+def test_queries_are_causal(oracle_mod, name):
+    """Changing the newest cached token changes only the newest query's
+    result; changing the token before it leaves position 0 of 3 alone and
+    changes positions 1 and 2."""
+    x = W.make_inputs(_q_shape(name, 3), seed=22)
+    out0, _ = oracle_mod.decode(x)
+    for back, unchanged in ((1, [0, 1]), (2, [0])):
+        kv = x["kv"].copy()
+        for b in range(x["shape"].batch):
+            page, slot = W.token_location(x, b, int(x["seq_lens"][b]) - back)
+            if x["shape"].latent:
+                kv[page, slot] = W.f32_to_bf16_bits(np.full(kv[page, slot].shape, 3.0, np.float32))
+            else:
+                kv[page, :, slot] = W.f32_to_bf16_bits(np.full(kv[page, :, slot].shape, 3.0, np.float32))
+        out1, _ = oracle_mod.decode(dict(x, kv=kv))
+        np.testing.assert_array_equal(out1[:, unchanged], out0[:, unchanged])
+        changed = [i for i in range(3) if i not in unchanged]
+        assert np.abs(out1[:, changed] - out0[:, changed]).max() > 1e-3
+
+
+def test_queries_match_a_masked_brute_force(oracle_mod):
+    """Tiny MLA with 3 query tokens against numpy softmax(QK^T + causal mask) V
+    over the gathered cache, all positions at once."""
+    s = W.WORKLOADS["mla"].replace(batch=1, num_q_heads=2, d_nope=8, d_rope=8, ctx=(7, 7), q_len=3,
+                                   page_size=64)
+    x = W.make_inputs(s, seed=23)
+    out, lse = oracle_mod.decode(x)
+    L = int(x["seq_lens"][0])
+    rows = np.stack([W.bf16_bits_to_f32(x["kv"][W.token_location(x, 0, j)]) for j in range(L)]).astype(np.float64)
+    qn = W.bf16_bits_to_f32(x["q_nope"][0]).astype(np.float64)     # [3][H][8]
+    qr = W.bf16_bits_to_f32(x["q_rope"][0]).astype(np.float64)
+    q = np.concatenate([qn, qr], axis=-1)                          # [3][H][16]
+    scores = np.einsum("ihd,jd->ihj", q, rows) * x["sm_scale"]
+    mask = np.arange(L)[None, :] <= (L - 3 + np.arange(3))[:, None]    # [3][L]
+    scores = np.where(mask[:, None, :], scores, -np.inf)
+    m = scores.max(-1, keepdims=True)
+    p = np.exp(scores - m)
+    z = p.sum(-1, keepdims=True)
+    ref = np.einsum("ihj,jd->ihd", p / z, rows[:, :8])
+    np.testing.assert_allclose(out[0], ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse[0], (m + np.log(z))[..., 0], rtol=1e-12, atol=1e-12)
