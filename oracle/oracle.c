@@ -70,6 +70,7 @@ typedef struct {
     double *out, *lse;
     int32_t nthreads, tid;
     int status;
+    int32_t branch_out;   /* MLRA: write the branch outputs side by side instead of their sum */
 } orc_job;
 
 /* Widen one input element to double (bf16 bits are the top half of a float). */
@@ -200,8 +201,11 @@ static void *worker(void *arg)
         double *dst = J->out + ((size_t)bi * nh + hi) * dn;
         if (s->variant == ORC_MLRA) {
             int R = s->num_kv;
-            for (int d = 0; d < dn; ++d)
-                dst[d] = 0.0;
+            if (J->branch_out)
+                dst = J->out + ((size_t)bi * nh + hi) * R * dn;
+            else
+                for (int d = 0; d < dn; ++d)
+                    dst[d] = 0.0;
             for (int r = 0; r < R; ++r) {
                 double l;
                 size_t q_row = ((size_t)b * H + h) * R + r;
@@ -209,8 +213,13 @@ static void *worker(void *arg)
                     J->status = -1;
                     goto done;
                 }
-                for (int d = 0; d < dn; ++d)
-                    dst[d] += o[d];
+                /* branch outputs side by side, or their sum */
+                for (int d = 0; d < dn; ++d) {
+                    if (J->branch_out)
+                        dst[(size_t)r * dn + d] = o[d];
+                    else
+                        dst[d] += o[d];
+                }
                 J->lse[((size_t)bi * nh + hi) * R + r] = l;
             }
         } else {
@@ -237,14 +246,15 @@ done:
  * Decode attention for the sequences listed in b_list (n_b of them) and the
  * heads listed in h_list (n_h of them; h_list = NULL means all H heads).
  * elem_type: 0 = inputs are bf16 bit patterns (uint16), 1 = inputs are double.
- * out: [n_b][n_h][d_nope] (MLRA: sum over branches); lse: [n_b][n_h] (MLRA
+ * out: [n_b][n_h][d_nope] (MLRA: sum over branches, or with branch_out the
+ * R branch outputs [n_b][n_h][R][d_nope]); lse: [n_b][n_h] (MLRA
  * [n_b][n_h][R]).  Returns 0, -1 for a page id outside the pool, -2 when out
  * of memory, -3 for an invalid shape.
  */
 int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const void *q_rope,
                const void *kv, const int32_t *block_table, const int32_t *seq_lens,
                double sm_scale, const int32_t *b_list, int32_t n_b, const int32_t *h_list,
-               int32_t n_h, double *out, double *lse, int32_t nthreads)
+               int32_t n_h, double *out, double *lse, int32_t nthreads, int32_t branch_out)
 {
     if (!s || s->variant < 0 || s->variant > 4 || s->num_kv <= 0 || s->num_q_heads <= 0 ||
         s->d_nope <= 0 || s->d_rope < 0 || s->page_size <= 0)
@@ -276,7 +286,7 @@ int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const 
     }
     for (int t = 0; t < nthreads; ++t) {
         orc_job J = {s, elem_type, q_nope, q_rope, kv, block_table, seq_lens, b_list, h_list,
-                     n_b, n_h, sm_scale, out, lse, nthreads, t, 0};
+                     n_b, n_h, sm_scale, out, lse, nthreads, t, 0, branch_out};
         jobs[t] = J;
     }
     int started = 0;

@@ -49,7 +49,7 @@ def _load():
         vp, i32p, dp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)
         lib.orc_decode.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int32, vp, vp, vp, i32p, i32p,
                                    ctypes.c_double, i32p, ctypes.c_int32, i32p, ctypes.c_int32, dp, dp,
-                                   ctypes.c_int32]
+                                   ctypes.c_int32, ctypes.c_int32]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, dp, dp, dp, dp]
         lib.orc_merge.restype = None
@@ -67,8 +67,9 @@ def _ptr(a, ctype):
 
 def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pages_per_seq,
          num_pages, paged, elem_type, q_nope, q_rope, kv, block_table, seq_lens, sm_scale,
-         b_list, nthreads, h_list=None):
+         b_list, nthreads, h_list=None, branch_out=False):
     lib = _load()
+    branch_out = bool(branch_out) and variant == "mlra"
     shp = _Shape(VARIANT_IDS[variant], batch, num_q_heads, num_kv, d_nope, d_rope, page_size,
                  max_pages_per_seq, num_pages, 1 if paged else 0)
     dt = np.uint16 if elem_type == 0 else np.float64
@@ -84,7 +85,7 @@ def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pag
     if h_list is not None:
         h_list = np.ascontiguousarray(h_list, dtype=np.int32)
     nh = num_q_heads if h_list is None else len(h_list)
-    out = np.zeros((nb, nh, d_nope), dtype=np.float64)
+    out = np.zeros((nb, nh, num_kv, d_nope) if branch_out else (nb, nh, d_nope), dtype=np.float64)
     lse_rows = nh * num_kv if variant == "mlra" else nh
     lse = np.zeros((nb, lse_rows), dtype=np.float64)
     rc = lib.orc_decode(ctypes.byref(shp), elem_type, q_nope.ctypes.data,
@@ -93,7 +94,7 @@ def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pag
                         float(sm_scale), _ptr(b_list, ctypes.c_int32), nb,
                         None if h_list is None else _ptr(h_list, ctypes.c_int32), nh,
                         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
-                        int(nthreads or default_threads()))
+                        int(nthreads or default_threads()), 1 if branch_out else 0)
     if rc != 0:
         raise RuntimeError(f"oracle failed with status {rc}")
     if variant == "mlra":
@@ -101,26 +102,29 @@ def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pag
     return out, lse
 
 
-def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None):
+def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None,
+           branch_out: bool = False):
     """fp64 decode attention of a workload dict (from ``workloads.make_inputs``).
 
     Returns ``(out, lse)``: out ``[n_b][n_h][d_nope]`` float64 (MLRA: the sum
-    over branches), lse ``[n_b][n_h]`` (MLRA ``[n_b][n_h][R]``), natural log.
+    over branches; with ``branch_out`` the R branch outputs ``[n_b][n_h][R][d_nope]``),
+    lse ``[n_b][n_h]`` (MLRA ``[n_b][n_h][R]``), natural log.
     ``b_list`` / ``h_list`` select sequences / heads (default: all).  With
     several query tokens per sequence (``shape.q_len`` = Q > 1) the results
     carry a query axis after the sequence axis: see ``decode_queries``.
     """
     s = inputs["shape"]
     if getattr(s, "q_len", 1) > 1:
-        return decode_queries(inputs, b_list, nthreads, sm_scale, h_list)
+        return decode_queries(inputs, b_list, nthreads, sm_scale, h_list, branch_out)
     scale = inputs["sm_scale"] if sm_scale is None else sm_scale
     return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
                 inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 0,
                 inputs["q_nope"], inputs["q_rope"], inputs["kv"], inputs["block_table"],
-                inputs["seq_lens"], scale, b_list, nthreads, h_list)
+                inputs["seq_lens"], scale, b_list, nthreads, h_list, branch_out)
 
 
-def decode_queries(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None):
+def decode_queries(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None,
+                   branch_out: bool = False):
     """Decode with Q > 1 query tokens per sequence (speculative or multi-token
     decode; the GLA page sets query length 1 against longer queries).
 
@@ -154,12 +158,13 @@ def decode_queries(inputs: dict, b_list=None, nthreads: int | None = None, sm_sc
     rows = dict(inputs, shape=s.replace(batch=B * Q, q_len=1, paged=True), q_nope=rows_q, q_rope=rows_qr,
                 seq_lens=rows_len, block_table=np.ascontiguousarray(rows_bt, dtype=np.int32))
     sel = (bs[:, None] * Q + np.arange(Q)).reshape(-1)
-    out, lse = decode(rows, b_list=sel, nthreads=nthreads, sm_scale=sm_scale, h_list=h_list)
+    out, lse = decode(rows, b_list=sel, nthreads=nthreads, sm_scale=sm_scale, h_list=h_list,
+                      branch_out=branch_out)
     return out.reshape((len(bs), Q) + out.shape[1:]), lse.reshape((len(bs), Q) + lse.shape[1:])
 
 
 def decode_f64(variant, num_kv, q_nope, q_rope, kv, seq_lens, sm_scale, block_table=None,
-               page_size=64, b_list=None, nthreads=None):
+               page_size=64, b_list=None, nthreads=None, branch_out=False):
     """Same computation on float64 arrays in the same layouts.
 
     ``q_nope`` is ``[B][H][d_nope]`` (MLRA ``[B][H][R][d_nope]``), ``kv`` is the
@@ -177,7 +182,7 @@ def decode_f64(variant, num_kv, q_nope, q_rope, kv, seq_lens, sm_scale, block_ta
         mpps = np.asarray(block_table).shape[1]
     return _run(variant, batch, H, num_kv, d_nope, d_rope, page_size, mpps, num_pages,
                 block_table is not None, 1, q_nope, q_rope, kv, block_table, seq_lens, sm_scale,
-                b_list, nthreads)
+                b_list, nthreads, None, branch_out)
 
 
 def merge(o_s: np.ndarray, lse_s: np.ndarray):
