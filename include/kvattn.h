@@ -98,7 +98,9 @@ enum kvattn_status {
 enum kvattn_device_error {
     KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1, /* block_table entry outside [0, num_pages): page skipped */
     KVATTN_DEVERR_SEQ_TOO_LONG = 2,      /* seq_lens[b] > max_seq_len: clamped to max_seq_len */
-    KVATTN_DEVERR_WAIT_TIMEOUT = 4       /* a bounded wait on an mbarrier ran out: tile skipped */
+    KVATTN_DEVERR_WAIT_TIMEOUT = 4,      /* a bounded wait on an mbarrier ran out: tile skipped */
+    KVATTN_DEVERR_POS_OUT_OF_RANGE = 8   /* kvattn_append_kv: a position outside the sequence's
+                                            pages: that token skipped */
 };
 
 /* Which decode kernel a plan uses. */
@@ -137,6 +139,10 @@ typedef struct {
     int32_t out_dtype;         /* kvattn_out_dtype */
     int32_t q_len;             /* query tokens per sequence, 1..64 (0 means 1); batch * q_len
                                   <= 65535 */
+    int32_t branch_out;        /* MLRA only (0 elsewhere): 1 = out holds the R normalised branch
+                                  outputs side by side, [B][Q][H][R][d_nope], instead of their
+                                  sum, for an up-projection with one W_UV block per branch
+                                  (kvattn_head_proj) */
 } kvattn_params;
 
 /* What kvattn_decode will launch for a problem (see kvattn_get_plan). */
@@ -263,6 +269,69 @@ int kvattn_decode_noalloc(int32_t variant, const kvattn_params *p, const void *q
 #define KVATTN_SELFTEST_MISSED_PHASE 256
 int kvattn_selftest_bounded_wait(int32_t *result, int32_t tries, void *stream);
 
+/*
+ * The steps either side of attention.
+ *
+ * kvattn_rope: rotary position embedding in place (MLA explainer section 2.2:
+ * the position branch's q^R and k^R are rotated; the pages print no formula,
+ * and this is the embedding's original form).  x is bf16 [rows][row_elems];
+ * in each row the slice [rot_offset, rot_offset + rot_dim) is taken as
+ * pairs (x[2i], x[2i+1]) and pair i is turned by the angle
+ * pos * rope_base^(-2i/rot_dim), pos = pos[row / rows_per_pos] (int32, any
+ * value; used as given).  Angle and turn in double precision, one rounding
+ * to bf16 (nearest even).  For the absorbed query of MLA/GLA (q_rope
+ * [B][Q][H][d_rope]): rows = B*Q*H, row_elems = rot_dim = d_rope,
+ * rows_per_pos = H, pos[B*Q] the query tokens' positions; MLRA rows carry R
+ * slices each (rows = B*Q*H*R, rows_per_pos = H*R).  rot_offset, rot_dim and
+ * row_elems even, rope_base > 1, x and pos 4-byte aligned; rows = 0 does
+ * nothing.  INVALID_ARG / MISALIGNED before anything is enqueued.
+ */
+int kvattn_rope(void *x, int32_t rows, int32_t row_elems, int32_t rot_offset, int32_t rot_dim,
+                int32_t rows_per_pos, const int32_t *pos, float rope_base, void *stream);
+
+/*
+ * kvattn_append_kv: write the newest tokens of each sequence into the paged
+ * cache decode reads (MLA explainer section 2.4: the compact latent is what
+ * the cache keeps).  p gives the cache geometry (batch, q_len = tokens per
+ * sequence, num_kv, d_nope, d_rope, max_pages_per_seq, num_pages; the other
+ * fields are checked as for decode).  new_kv, bf16, caller-owned:
+ *   latent variants  [B][Q][num_kv*d_nope + d_rope], [c_0 | ... | k^R] with
+ *                    k^R not yet rotated;
+ *   GQA/MQA          [B][Q][2][num_kv][d_nope], K then V.
+ * pos int32 [B][Q]: the cache position of each token (slot pos % 64 of page
+ * block_table[b][pos / 64]; block_table NULL = contiguous, as in decode).
+ * rope_base > 1 rotates k^R (latent) or every K head (GQA/MQA) at its
+ * position on the way in, exactly as kvattn_rope does; rope_base = 0 stores
+ * the rows as given.  Latent parts and V are copied bit for bit.  A position
+ * outside [0, max_pages_per_seq * 64) sets KVATTN_DEVERR_POS_OUT_OF_RANGE, a
+ * page id outside [0, num_pages) KVATTN_DEVERR_PAGE_OUT_OF_RANGE, in
+ * *device_error (int32 device word, may be NULL), and that token is skipped.
+ * new_kv and kv_cache 16-byte aligned.  Seq_lens are not touched: the caller
+ * counts the new tokens in before the next decode.
+ */
+int kvattn_append_kv(int32_t variant, const kvattn_params *p, const void *new_kv, const int32_t *pos,
+                     const int32_t *block_table, void *kv_cache, float rope_base, int32_t *device_error,
+                     void *stream);
+
+/*
+ * kvattn_head_proj: y[r][h][:] = x[r][h][:] @ w[h] for every row r and head h,
+ * bf16 inputs, fp32 accumulation on the tensor cores, y bf16 (nearest even)
+ * or fp32 (out_dtype).  x [rows][heads][k], w [heads][k][n], y
+ * [rows][heads][n], row-major, 16-byte aligned; k and n multiples of 64.
+ *   Query absorption (MLRA page, MLA paragraph: W_UK folded into the query):
+ *     x = q^C [B*Q][H][d_h], w = W_UK [H][d_h][d_c] (per MLRA head the R
+ *     branch blocks side by side, n = R*d_c), y = q_nope for decode.
+ *   Up-projection (MLA explainer section 2.3: outputs weight c W_UV):
+ *     x = decode's out [B*Q][H][d_c] (MLRA with branch_out: [B*Q][H][R*d_c]),
+ *     w = W_UV [H][d_c][d_v] (MLRA: the R branch blocks stacked, k = R*d_c,
+ *     so the branch sum of "moving the sum outside" is part of the
+ *     contraction), y the attention output per head.
+ * A wait that runs out sets KVATTN_DEVERR_WAIT_TIMEOUT in *device_error (may
+ * be NULL).  rows = 0 does nothing.
+ */
+int kvattn_head_proj(const void *x, const void *w, void *y, int32_t out_dtype, int32_t rows, int32_t heads,
+                     int32_t k, int32_t n, int32_t *device_error, void *stream);
+
 /* Copy the device error word to *code (0 = none, else kvattn_device_error
  * bits).  Synchronises `stream`.  Returns KVATTN_ERR_CUDA if the copy
  * failed. */
@@ -271,7 +340,9 @@ int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code);
 /* Static, human-readable name of a status code. */
 const char *kvattn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 200 (kvattn_params carries q_len). */
+/* Library ABI version (major * 100 + minor): 201 (kvattn_params carries q_len and
+ * branch_out; the steps either side: kvattn_rope, kvattn_append_kv,
+ * kvattn_head_proj). */
 int kvattn_version(void);
 
 #ifdef __cplusplus

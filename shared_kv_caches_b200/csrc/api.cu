@@ -29,6 +29,8 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
         return KVATTN_ERR_INVALID_ARG;
     if (p->q_len < 0)
         return KVATTN_ERR_INVALID_ARG;
+    if (p->branch_out != 0 && (p->branch_out != 1 || variant != KVATTN_MLRA))
+        return KVATTN_ERR_INVALID_ARG;
     const int q_len = p->q_len > 0 ? p->q_len : 1;
     if (q_len > kMaxQueryLen || (long long)p->batch * q_len > 65535 || p->num_q_heads > 65535)
         return KVATTN_ERR_UNSUPPORTED;
@@ -73,6 +75,7 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
     pr->max_seq_len = p->max_seq_len;
     pr->out_dtype = p->out_dtype;
     pr->paged = true;
+    pr->branch_out = p->branch_out != 0;
     return KVATTN_OK;
 }
 
@@ -218,6 +221,8 @@ int sm_count()
     return cached[dev];
 }
 
+int validate_params(int32_t variant, const kvattn_params *p, Problem *pr) { return validate(variant, p, pr); }
+
 int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
                   const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
                   float sm_scale, const void *out, const float *lse, const void *workspace,
@@ -243,7 +248,7 @@ int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, c
 
 using namespace kvattn;
 
-extern "C" int kvattn_version(void) { return 200; }
+extern "C" int kvattn_version(void) { return 201; }
 
 extern "C" const char *kvattn_status_string(int status)
 {
@@ -382,6 +387,12 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     c.HU = pr.HU;
     c.num_splits = pl.pub.num_splits;
     c.mlra = pr.mlra;
+    if (pr.branch_out) {
+        // every (head, branch) row merged on its own and written in place:
+        // out[b][h][r] is row b * H * R + h * R + r, as the partial rows are
+        c.mlra = 0;
+        c.H = pr.HU;
+    }
     c.out_fp32 = pr.out_dtype == KVATTN_OUT_FP32;
     if (launch_combine(c, s) != cudaSuccess)
         return KVATTN_ERR_CUDA;

@@ -28,6 +28,7 @@ struct Problem {
     int HU;            // partial rows per sequence: H, or H*R for MLRA
     int mpps, num_pages, max_seq_len, out_dtype;
     bool latent, mlra, paged;
+    bool branch_out;   // MLRA: the R branch outputs side by side instead of their sum
 };
 
 // Arguments of every decode kernel.  Partial results go to the workspace as
@@ -182,6 +183,8 @@ int sm_count();
 // Argument checks shared by every decode entry point: the problem, the
 // pointers and their alignment, sm_scale.  Returns a kvattn_status; nothing
 // is enqueued.
+// Shape checks of kvattn_params (the Problem every entry point works from).
+int validate_params(int32_t variant, const kvattn_params *p, Problem *pr);
 int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, const void *q_rope,
                   const void *kv_cache, const int32_t *block_table, const int32_t *seq_lens,
                   float sm_scale, const void *out, const float *lse, const void *workspace,

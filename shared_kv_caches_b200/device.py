@@ -61,6 +61,17 @@ class DeviceProblem:
                          self.lse if lse is None else lse,
                          self.workspace, stream, events)
 
+    def append_kv(self, new_kv, pos, rope_base, device_error=None, stream=None):
+        """Write new token rows into this problem's cache (kvattn_append_kv)."""
+        import torch
+        st = K.kvattn_append_kv(self.variant, self.params, new_kv.data_ptr(), pos.data_ptr(),
+                                None if self.block_table is None else self.block_table.data_ptr(),
+                                self.kv.data_ptr(), rope_base,
+                                None if device_error is None else device_error.data_ptr(),
+                                torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream)
+        if st:
+            raise K.KvattnError(st, "kvattn_append_kv")
+
     def plan_kernel_name(self) -> str:
         return K.KERNEL_NAMES.get(int(self.plan.kernel), str(self.plan.kernel))
 

@@ -31,19 +31,21 @@ KVATTN_ERR_CUDA = -5
 KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1
 KVATTN_DEVERR_SEQ_TOO_LONG = 2
 KVATTN_DEVERR_WAIT_TIMEOUT = 4
+KVATTN_DEVERR_POS_OUT_OF_RANGE = 8
 KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc", 4: "latent_pair"}
 KVATTN_SELFTEST_MISSED_PHASE = 256
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
            "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
-           "kvattn_status_string", "kvattn_version", "kvattn_selftest_bounded_wait")
+           "kvattn_status_string", "kvattn_version", "kvattn_selftest_bounded_wait", "kvattn_rope",
+           "kvattn_append_kv", "kvattn_head_proj")
 KVATTN_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class kvattn_params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "num_q_heads", "num_kv", "d_nope", "d_rope", "page_size", "max_pages_per_seq",
-        "num_pages", "max_seq_len", "num_splits", "out_dtype", "q_len")]
+        "num_pages", "max_seq_len", "num_splits", "out_dtype", "q_len", "branch_out")]
 
 
 class kvattn_plan(ctypes.Structure):
@@ -85,19 +87,24 @@ def load():
     lib.kvattn_status_string.restype = ctypes.c_char_p
     lib.kvattn_version.argtypes = []
     lib.kvattn_selftest_bounded_wait.argtypes = [vp, i32, vp]
+    lib.kvattn_rope.argtypes = [vp, i32, i32, i32, i32, i32, vp, ctypes.c_float, vp]
+    lib.kvattn_append_kv.argtypes = [i32, P, vp, vp, vp, vp, ctypes.c_float, vp, vp]
+    lib.kvattn_head_proj.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     for name in ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
                  "kvattn_decode_timed", "kvattn_decode_noalloc", "kvattn_get_device_error",
-                 "kvattn_version", "kvattn_selftest_bounded_wait"):
+                 "kvattn_version", "kvattn_selftest_bounded_wait", "kvattn_rope", "kvattn_append_kv",
+                 "kvattn_head_proj"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
 
 
 def make_params(batch, num_q_heads, num_kv, d_nope, d_rope, max_pages_per_seq, num_pages,
-                max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64, q_len=1) -> kvattn_params:
+                max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64, q_len=1,
+                branch_out=0) -> kvattn_params:
     return kvattn_params(int(batch), int(num_q_heads), int(num_kv), int(d_nope), int(d_rope),
                          int(page_size), int(max_pages_per_seq), int(num_pages), int(max_seq_len),
-                         int(num_splits), int(out_dtype), int(q_len))
+                         int(num_splits), int(out_dtype), int(q_len), int(branch_out))
 
 
 def kvattn_version() -> int:
@@ -178,7 +185,7 @@ def params_for(shape, max_pages_per_seq, num_pages, max_seq_len, num_splits=0) -
     return make_params(shape.batch, shape.num_q_heads, shape.num_kv, shape.d_nope, shape.d_rope,
                        max_pages_per_seq, num_pages, max_seq_len, num_splits,
                        KVATTN_OUT_FP32 if shape.out_dtype == "fp32" else KVATTN_OUT_BF16,
-                       shape.page_size, shape.q_len)
+                       shape.page_size, shape.q_len, 1 if getattr(shape, "branch_out", False) else 0)
 
 
 def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, sm_scale, out, lse,
@@ -200,3 +207,50 @@ def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, s
         st = kvattn_decode_timed(*args, [None if e is None else e.cuda_event for e in events])
     if st:
         raise KvattnError(st, "kvattn_decode")
+
+
+# ------------------------------------------------- the steps either side
+
+def kvattn_rope(x, rows, row_elems, rot_offset, rot_dim, rows_per_pos, pos, rope_base, stream=0) -> int:
+    return load().kvattn_rope(x, int(rows), int(row_elems), int(rot_offset), int(rot_dim), int(rows_per_pos),
+                              pos, float(rope_base), stream)
+
+
+def kvattn_append_kv(variant, params, new_kv, pos, block_table, kv_cache, rope_base, device_error=None,
+                     stream=0) -> int:
+    return load().kvattn_append_kv(int(variant), ctypes.byref(params), new_kv, pos, block_table, kv_cache,
+                                   float(rope_base), device_error, stream)
+
+
+def kvattn_head_proj(x, w, y, out_dtype, rows, heads, k, n, device_error=None, stream=0) -> int:
+    return load().kvattn_head_proj(x, w, y, int(out_dtype), int(rows), int(heads), int(k), int(n),
+                                   device_error, stream)
+
+
+def rope_tensor(x, pos, rot_offset, rot_dim, rope_base, rows_per_pos):
+    """In-place RoPE on a contiguous bf16 tensor whose last axis is the row
+    (argument marshalling only; the rotation runs in kvattn_rope)."""
+    import torch
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and pos.dtype == torch.int32
+    row_elems = x.shape[-1]
+    rows = x.numel() // row_elems
+    st = kvattn_rope(_ptr(x), rows, row_elems, rot_offset, rot_dim, rows_per_pos, _ptr(pos), rope_base,
+                     torch.cuda.current_stream(x.device).cuda_stream)
+    if st:
+        raise KvattnError(st, "kvattn_rope")
+
+
+def head_proj_tensor(x, w, out_fp32=False):
+    """y[r, h] = x[r, h] @ w[h] for bf16 x [rows][H][k] and w [H][k][n] on the
+    device (kvattn_head_proj); returns y [rows][H][n]."""
+    import torch
+    assert x.dtype == torch.bfloat16 and w.dtype == torch.bfloat16 and x.is_contiguous() and w.is_contiguous()
+    rows, heads, k = x.shape
+    n = w.shape[2]
+    assert w.shape[:2] == (heads, k)
+    y = torch.empty((rows, heads, n), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=x.device)
+    st = kvattn_head_proj(_ptr(x), _ptr(w), _ptr(y), KVATTN_OUT_FP32 if out_fp32 else KVATTN_OUT_BF16, rows,
+                          heads, k, n, None, torch.cuda.current_stream(x.device).cuda_stream)
+    if st:
+        raise KvattnError(st, "kvattn_head_proj")
+    return y

@@ -71,6 +71,7 @@ class Shape:
     sm_scale: float | None = None
     input_scale: float = 1.0
     q_len: int = 1          # query tokens per sequence (the newest q_len cached tokens)
+    branch_out: bool = False  # MLRA: the branch outputs side by side instead of their sum
 
     @property
     def variant_id(self) -> int:
@@ -131,6 +132,8 @@ class Shape:
         return self._rows() + (self.num_q_heads, self.d_rope)
 
     def out_shape(self) -> tuple:
+        if self.branch_out:
+            return self._rows() + (self.num_q_heads, self.num_kv, self.d_nope)
         return self._rows() + (self.num_q_heads, self.d_nope)
 
     def lse_shape(self) -> tuple:
@@ -296,3 +299,47 @@ def token_location(inputs: dict, b: int, j: int) -> tuple:
     if bt is None:
         return b * inputs["max_pages_per_seq"] + j // ps, j % ps
     return int(bt[b, j // ps]), j % ps
+
+
+# The steps either side of attention: what a decode step gets before the
+# cache and the absorbed query exist.  Head width d_h and value width d_v are
+# 128 (the per-head widths of the pages' MLA-family models); the position
+# base is 10000.
+HEAD_DIM = 128
+ROPE_BASE = 10000.0
+
+
+def step_widths(shape: Shape) -> tuple:
+    """(k of the absorption = d_h, latent columns each head reads = n of the
+    absorption and k of the up-projection, d_v)."""
+    per_head = shape.num_kv * shape.d_nope if shape.variant == "mlra" else shape.d_nope
+    return HEAD_DIM, per_head, HEAD_DIM
+
+
+def make_step_inputs(shape: Shape, seed: int = 0, seq_lens=None) -> dict:
+    """Seeded inputs of the steps around decode for a latent ``shape``:
+
+    q_c     bf16 [B][Q][H][d_h]            semantic query before absorption
+    w_uk    bf16 [H][d_h][n_abs]            per-head key up-projection (MLRA: the R
+                                            branch blocks side by side, n_abs = R d_c)
+    w_uv    bf16 [H][n_abs][d_v]            per-head value up-projection (MLRA: the R
+                                            branch blocks stacked)
+    new_kv  bf16 [B][Q][row]                the newest tokens' rows, k^R not yet rotated
+    pos     int32 [B][Q]                    their positions: seq_lens[b] - Q + i
+    plus everything ``make_inputs`` returns (the cache, the raw q_rope, ...).
+    Weights are N(0, 1/fan_in) so the projections stay O(1)."""
+    if not shape.latent:
+        raise ValueError("the absorbed steps concern the latent variants")
+    x = make_inputs(shape, seed, seq_lens=seq_lens)
+    rng = np.random.default_rng(seed + 7919)
+    d_h, n_abs, d_v = step_widths(shape)
+    rows = shape._rows()
+    x["q_c"] = _normal_bf16(rng, rows + (shape.num_q_heads, d_h), shape.input_scale)
+    x["w_uk"] = _normal_bf16(rng, (shape.num_q_heads, d_h, n_abs), 1.0 / math.sqrt(d_h))
+    x["w_uv"] = _normal_bf16(rng, (shape.num_q_heads, n_abs, d_v), 1.0 / math.sqrt(n_abs))
+    q = shape.q_len
+    x["new_kv"] = _normal_bf16(rng, (shape.batch, q, shape.row_elems), shape.input_scale)
+    lens = np.asarray(x["seq_lens"], dtype=np.int64)
+    x["pos"] = np.maximum(lens[:, None] - q + np.arange(q)[None, :], 0).astype(np.int32)
+    x["rope_base"] = ROPE_BASE
+    return x
