@@ -32,6 +32,10 @@ buffers, the oracle timed on the host cores for the headline problem (rank 0,
 N = 1), SM clocks sampled during the timed regions, and how many of the
 library's kernels ran in the headline's timed region.
 
+``steps`` times the steps either side of attention at the benchmark shapes
+(query absorption and up-projection per head, the query RoPE, the cache
+append), each an event-timed call against its algorithmic HBM bytes.
+
 ``--impl reference`` times the fp64 CPU oracle (the reference arm) on the
 headline problem, each step a bounded sample of it, and prints the same line
 with ``"impl": "reference"``.
@@ -68,6 +72,7 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--splits", type=int, default=0, help="force parts per context (0: library choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-steps", action="store_true", help="skip the steps either side of attention")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     a = ap.parse_args(argv)
     if a.warmup < 3:
@@ -279,6 +284,86 @@ def measure(names, args, dev, world, peaks, flush, workload_label, want_inputs=F
     return out
 
 
+# The steps either side of attention at the benchmark shapes (rows = the
+# problem's batch x query tokens, H = 128 heads): query absorption
+# (W_UK, d_h = 128 -> the latent columns a head reads), the up-projection
+# (W_UV, those columns -> d_v = 128; MLRA with its four branch blocks
+# stacked), the query RoPE and the cache append of the newest tokens.
+STEP_OPS = {
+    "mla_absorb": ("proj", 64, 128, 128, 512),
+    "mla_up": ("proj", 64, 128, 512, 128),
+    "gla_absorb": ("proj", 64, 128, 128, 256),
+    "gla_up": ("proj", 64, 128, 256, 128),
+    "mlra_b8_absorb": ("proj", 8, 128, 128, 512),
+    "mlra_b8_up": ("proj", 8, 128, 512, 128),
+    "mla_rope_q": ("rope", 64 * 128, 64),
+    "mla_append": ("append", "mla"),
+}
+
+
+def measure_steps(args, dev, peaks, flush):
+    """Event-timed calls of each step op (L2 flushed between calls) with its
+    algorithmic HBM bytes; all of them are bound by HBM."""
+    import numpy as np
+    import torch
+
+    from shared_kv_caches_b200 import kvattn as K
+    from shared_kv_caches_b200 import workloads as W
+    from shared_kv_caches_b200.device import DeviceProblem
+
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    stream = lambda: torch.cuda.current_stream(dev).cuda_stream
+    out = {}
+    for name, spec in STEP_OPS.items():
+        kind = spec[0]
+        if kind == "proj":
+            _, rows, heads, k, n = spec
+            x = torch.randn((rows, heads, k), generator=gen, device=dev).to(torch.bfloat16)
+            w = (torch.randn((heads, k, n), generator=gen, device=dev) / k ** 0.5).to(torch.bfloat16)
+            y = torch.empty((rows, heads, n), dtype=torch.bfloat16, device=dev)
+            nbytes = 2 * (x.numel() + w.numel() + y.numel())
+            call = lambda: K.kvattn_head_proj(x.data_ptr(), w.data_ptr(), y.data_ptr(), K.KVATTN_OUT_BF16, rows,
+                                              heads, k, n, None, stream())
+            what = f"y[{rows}][{heads}][{n}] = x[{rows}][{heads}][{k}] W[{heads}][{k}][{n}]"
+        elif kind == "rope":
+            _, rows, rd = spec
+            q = torch.randn((rows, rd), generator=gen, device=dev).to(torch.bfloat16)
+            pos = torch.randint(0, 1 << 15, (rows // 128,), generator=gen, device=dev, dtype=torch.int32)
+            nbytes = 2 * 2 * q.numel() + 4 * pos.numel()
+            call = lambda: K.kvattn_rope(q.data_ptr(), rows, rd, 0, rd, 128, pos.data_ptr(), W.ROPE_BASE, stream())
+            what = f"q_rope[{rows // 128}][128][{rd}] turned in place"
+        else:
+            s = W.WORKLOADS[spec[1]]
+            xin = W.make_step_inputs(s.replace(ctx=(256, 512)), seed=args.seed)
+            prob = DeviceProblem(xin, dev)
+            new = torch.from_numpy(np.ascontiguousarray(xin["new_kv"]).view(np.int16)).view(torch.bfloat16).to(dev)
+            pos = torch.from_numpy(xin["pos"]).to(dev)
+            nbytes = 2 * 2 * new.numel() + 4 * pos.numel() + 4 * s.batch
+            call = lambda: K.kvattn_append_kv(prob.variant, prob.params, new.data_ptr(), pos.data_ptr(),
+                                              prob.block_table.data_ptr(), prob.kv.data_ptr(), W.ROPE_BASE, None,
+                                              stream())
+            what = f"{s.batch} new [{s.row_elems}] rows into the paged cache, k^R turned"
+        for _ in range(args.warmup):
+            if call():
+                raise SystemExit(f"step op {name} refused")
+            flush.zero_()
+        n_t = min(args.steps, 50)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_t)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record()
+            call()
+            b.record()
+            flush.zero_()
+        torch.cuda.synchronize()
+        us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"op": what, "us": round(us, 2), "bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
+                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    torch.cuda.empty_cache()
+    return out
+
+
 def dist_rank():
     return int(os.environ.get("RANK", "0"))
 
@@ -356,6 +441,8 @@ def run_ours(args, rank, world, local):
                                                      "hbm_gbs", "kernels_us", "roofline", "e2e",
                                                      "gpu_launches")}
             for r in results}
+    if args.workload == "suite" and world == 1 and not args.no_steps:
+        line["steps"] = measure_steps(args, dev, peaks, flush)
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if world > 1:
