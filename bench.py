@@ -12,7 +12,8 @@ ragged contexts drawn uniformly from [4096, 32768] on a paged 64-token bf16
 cache with a permuted block table), the largest problem that fits one GPU;
 ``suite`` carries the same figures for GQA, MFA, GLA-2 and the four MLRA-4
 shapes.  ``--workload NAME`` times one problem (or ``gqa+mfa``, the GQA and
-MFA layers together as one step).
+MFA layers together as one step); ``--workload steps`` only the steps either
+side of attention.
 
 A step is one decode call of a problem (split pass + combine pass) over one
 batch of seeded synthetic input that is already resident in HBM.
@@ -34,7 +35,8 @@ library's kernels ran in the headline's timed region.
 
 ``steps`` times the steps either side of attention at the benchmark shapes
 (query absorption and up-projection per head, the query RoPE, the cache
-append), each an event-timed call against its algorithmic HBM bytes.
+append): calls back to back over input replicas larger than L2, against each
+op's algorithmic HBM bytes.
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm) on the
 headline problem, each step a bounded sample of it, and prints the same line
@@ -302,8 +304,11 @@ STEP_OPS = {
 
 
 def measure_steps(args, dev, peaks, flush):
-    """Event-timed calls of each step op (L2 flushed between calls) with its
-    algorithmic HBM bytes; all of them are bound by HBM."""
+    """Throughput of each step op as a model issues them, back to back on one
+    stream: K calls cycle through enough replicas of the op's inputs (and
+    outputs) to hold over 300 MB, so no call finds its operands in the 126 MB
+    L2; one event pair around the K calls.  Against the op's algorithmic HBM
+    bytes; all of them are bound by HBM."""
     import numpy as np
     import torch
 
@@ -312,55 +317,61 @@ def measure_steps(args, dev, peaks, flush):
     from shared_kv_caches_b200.device import DeviceProblem
 
     gen = torch.Generator(device=dev).manual_seed(args.seed)
-    stream = lambda: torch.cuda.current_stream(dev).cuda_stream
+    st = torch.cuda.current_stream(dev).cuda_stream
+    span = 300 << 20
     out = {}
     for name, spec in STEP_OPS.items():
         kind = spec[0]
         if kind == "proj":
             _, rows, heads, k, n = spec
-            x = torch.randn((rows, heads, k), generator=gen, device=dev).to(torch.bfloat16)
-            w = (torch.randn((heads, k, n), generator=gen, device=dev) / k ** 0.5).to(torch.bfloat16)
-            y = torch.empty((rows, heads, n), dtype=torch.bfloat16, device=dev)
-            nbytes = 2 * (x.numel() + w.numel() + y.numel())
-            call = lambda: K.kvattn_head_proj(x.data_ptr(), w.data_ptr(), y.data_ptr(), K.KVATTN_OUT_BF16, rows,
-                                              heads, k, n, None, stream())
+            nbytes = 2 * (rows * heads * k + heads * k * n + rows * heads * n)
+            reps = max(2, -(-span // nbytes))
+            xs = [torch.randn((rows, heads, k), generator=gen, device=dev).to(torch.bfloat16) for _ in range(reps)]
+            ws = [(torch.randn((heads, k, n), generator=gen, device=dev) / k ** 0.5).to(torch.bfloat16)
+                  for _ in range(reps)]
+            ys = [torch.empty((rows, heads, n), dtype=torch.bfloat16, device=dev) for _ in range(reps)]
+            call = lambda i: K.kvattn_head_proj(xs[i].data_ptr(), ws[i].data_ptr(), ys[i].data_ptr(),
+                                                K.KVATTN_OUT_BF16, rows, heads, k, n, None, st)
             what = f"y[{rows}][{heads}][{n}] = x[{rows}][{heads}][{k}] W[{heads}][{k}][{n}]"
         elif kind == "rope":
             _, rows, rd = spec
-            q = torch.randn((rows, rd), generator=gen, device=dev).to(torch.bfloat16)
+            nbytes = 2 * 2 * rows * rd + 4 * (rows // 128)
+            reps = max(2, -(-span // nbytes))
+            qs = [torch.randn((rows, rd), generator=gen, device=dev).to(torch.bfloat16) for _ in range(reps)]
             pos = torch.randint(0, 1 << 15, (rows // 128,), generator=gen, device=dev, dtype=torch.int32)
-            nbytes = 2 * 2 * q.numel() + 4 * pos.numel()
-            call = lambda: K.kvattn_rope(q.data_ptr(), rows, rd, 0, rd, 128, pos.data_ptr(), W.ROPE_BASE, stream())
+            call = lambda i: K.kvattn_rope(qs[i].data_ptr(), rows, rd, 0, rd, 128, pos.data_ptr(), W.ROPE_BASE, st)
             what = f"q_rope[{rows // 128}][128][{rd}] turned in place"
         else:
-            s = W.WORKLOADS[spec[1]]
-            xin = W.make_step_inputs(s.replace(ctx=(256, 512)), seed=args.seed)
+            s = W.WORKLOADS[spec[1]].replace(ctx=(4096, 4096))
+            xin = W.make_step_inputs(s, seed=args.seed)
             prob = DeviceProblem(xin, dev)
             new = torch.from_numpy(np.ascontiguousarray(xin["new_kv"]).view(np.int16)).view(torch.bfloat16).to(dev)
-            pos = torch.from_numpy(xin["pos"]).to(dev)
-            nbytes = 2 * 2 * new.numel() + 4 * pos.numel() + 4 * s.batch
-            call = lambda: K.kvattn_append_kv(prob.variant, prob.params, new.data_ptr(), pos.data_ptr(),
-                                              prob.block_table.data_ptr(), prob.kv.data_ptr(), W.ROPE_BASE, None,
-                                              stream())
+            nbytes = 2 * 2 * new.numel() + 4 * s.batch + 4 * s.batch
+            # replicas: the same rows written at 4096 different positions of
+            # every sequence (each call writes other cache lines)
+            reps = 4096
+            pos = [torch.full((s.batch, 1), i, dtype=torch.int32, device=dev) for i in range(reps)]
+            call = lambda i: K.kvattn_append_kv(prob.variant, prob.params, new.data_ptr(), pos[i].data_ptr(),
+                                                prob.block_table.data_ptr(), prob.kv.data_ptr(), W.ROPE_BASE,
+                                                None, st)
             what = f"{s.batch} new [{s.row_elems}] rows into the paged cache, k^R turned"
-        for _ in range(args.warmup):
-            if call():
+        for i in range(max(args.warmup, 3)):
+            if call(i % reps):
                 raise SystemExit(f"step op {name} refused")
-            flush.zero_()
-        n_t = min(args.steps, 50)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_t)]
+        flush.zero_()
+        n_t = max(args.steps, reps)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        for a, b in evs:
-            a.record()
-            call()
-            b.record()
-            flush.zero_()
+        a.record()
+        for i in range(n_t):
+            call(i % reps)
+        b.record()
         torch.cuda.synchronize()
-        us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+        us = a.elapsed_time(b) * 1e3 / n_t
         gbs = nbytes / (us * 1e-6) / 1e9
         out[name] = {"op": what, "us": round(us, 2), "bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
-                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-    torch.cuda.empty_cache()
+                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": n_t, "replicas": reps}
+        torch.cuda.empty_cache()
     return out
 
 
@@ -402,6 +413,16 @@ def run_ours(args, rank, world, local):
     sampler = BU.ClockSampler(bus_id=bus).start()
     time.sleep(0.3)
 
+    if args.workload == "steps":
+        # the steps either side of attention alone (for profiling them)
+        line = {"metric": "step_ops_us", "impl": "ours", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "steps_ops": measure_steps(args, dev, peaks, flush)}
+        sampler.stop()
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     groups = [(n,) for n in SUITE] if args.workload == "suite" else [problem_names(args.workload)]
     label = (lambda g: g[0]) if args.workload == "suite" else (lambda g: args.workload)
     cpu = None

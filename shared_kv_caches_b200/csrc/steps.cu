@@ -129,14 +129,15 @@ constexpr int kHpChunk = 64;                       // contraction elements per s
 constexpr int kHpXBytes = 128 * kHpChunk * 2;      // 128 rows x 64 (16 KB)
 constexpr int kHpWBox = kHpChunk * 64 * 2;         // 64 contraction rows x 64 columns (8 KB)
 
+// Shared memory of a head-projection CTA with `stages` ring slots (only as
+// many as the contraction has chunks, so short contractions fit two CTAs on
+// an SM): the x tiles, then the W tiles, then the barriers.
 template <int NT>
-struct HpSmem {
-    unsigned char x[kHpStages][kHpXBytes];
-    unsigned char w[kHpStages][NT / 64][kHpWBox];
-    uint64_t full[kHpStages];
-    uint64_t empty[kHpStages];
-    uint64_t done;
-    uint32_t tmem;
+struct HpLayout {
+    static constexpr int kWStage = (NT / 64) * kHpWBox;
+    __host__ __device__ static size_t w_off(int stages) { return (size_t)stages * kHpXBytes; }
+    __host__ __device__ static size_t bar_off(int stages) { return w_off(stages) + (size_t)stages * kWStage; }
+    __host__ __device__ static size_t bytes(int stages) { return bar_off(stages) + (2 * stages + 2) * 8; }
 };
 
 template <int NT>
@@ -151,36 +152,42 @@ constexpr uint32_t hp_tmem_cols()
 // i.e. rows m0 + 32w ..).  Rows past `rows` are zero-filled by TMA and not
 // stored.
 template <int NT>
-__global__ void __launch_bounds__(kHpThreads, 1)
+__global__ void __launch_bounds__(kHpThreads)
     head_proj_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, void *y,
-                     int out_fp32, int rows, int heads, int k, int n, int32_t *err)
+                     int out_fp32, int rows, int heads, int k, int n, int stages, int32_t *err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    HpSmem<NT> &S = *reinterpret_cast<HpSmem<NT> *>(smem_raw);
+    using Lay = HpLayout<NT>;
+    unsigned char *xs = smem_raw;                                  // [stages][kHpXBytes]
+    unsigned char *ws = smem_raw + Lay::w_off(stages);             // [stages][NT / 64][kHpWBox]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw + Lay::bar_off(stages));
+    uint64_t *empty = full + stages;
+    uint64_t *done = empty + stages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x, n0 = blockIdx.y * NT, m0 = blockIdx.z * 128;
     const int chunks = k / kHpChunk;
     constexpr uint32_t kCols = hp_tmem_cols<NT>();
-    constexpr uint32_t kStageTx = kHpXBytes + (NT / 64) * kHpWBox;
+    constexpr uint32_t kStageTx = kHpXBytes + Lay::kWStage;
     if (smem_u32(smem_raw) & 1023u) {
         if (threadIdx.x == 0 && err)
             atomicOr(err, KVATTN_DEVERR_WAIT_TIMEOUT);
         return;
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kHpStages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1);
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        mbar_init(&S.done, 1);
+        mbar_init(done, 1);
         fence_mbar_init();
     }
     if (warp == 0)
-        tmem_alloc(&S.tmem, kCols);
+        tmem_alloc(tmem_slot, kCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tacc = S.tmem;
+    const uint32_t tacc = *tmem_slot;
     bool ok = true;
 
     if (warp == 0) {
@@ -189,22 +196,23 @@ __global__ void __launch_bounds__(kHpThreads, 1)
             prefetch_tmap(&wmap);
             int issued = 0;
             for (int c = 0; c < chunks; ++c) {
-                const int st = c % kHpStages;
-                if (c >= kHpStages && !mbar_wait(&S.empty[st], ((c / kHpStages) - 1) & 1)) {
+                const int st = c % stages;
+                if (c >= stages && !mbar_wait(&empty[st], ((c / stages) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&S.full[st], kStageTx);
-                tma_load_3d(S.x[st], &xmap, c * kHpChunk, h, m0, &S.full[st]);
+                mbar_arrive_expect_tx(&full[st], kStageTx);
+                tma_load_3d(xs + (size_t)st * kHpXBytes, &xmap, c * kHpChunk, h, m0, &full[st]);
 #pragma unroll
                 for (int b = 0; b < NT / 64; ++b)
-                    tma_load_2d(S.w[st][b], &wmap, n0 + 64 * b, h * k + c * kHpChunk, &S.full[st]);
+                    tma_load_2d(ws + (size_t)st * Lay::kWStage + b * kHpWBox, &wmap, n0 + 64 * b,
+                                h * k + c * kHpChunk, &full[st]);
                 issued = c + 1;
             }
             // every copy started here has landed before the CTA can exit
-            for (int st = 0; st < kHpStages && st < issued; ++st) {
-                const int cl = st + ((issued - 1 - st) / kHpStages) * kHpStages;
-                if (!mbar_wait(&S.full[st], (cl / kHpStages) & 1))
+            for (int st = 0; st < stages && st < issued; ++st) {
+                const int cl = st + ((issued - 1 - st) / stages) * stages;
+                if (!mbar_wait(&full[st], (cl / stages) & 1))
                     ok = false;
             }
             if (!ok && err)
@@ -213,34 +221,34 @@ __global__ void __launch_bounds__(kHpThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         constexpr uint32_t idesc = idesc_bf16_f32(128, NT, false, true);
-        const uint64_t xdesc0 = smem_desc(smem_u32(S.x[0]), 16, 1024, 2);          // K-major rows of x
-        const uint64_t wdesc0 = smem_desc(smem_u32(S.w[0][0]), kHpWBox, 1024, 2);  // N-major rows of W
+        const uint64_t xdesc0 = smem_desc(smem_u32(xs), 16, 1024, 2);          // K-major rows of x
+        const uint64_t wdesc0 = smem_desc(smem_u32(ws), kHpWBox, 1024, 2);     // N-major rows of W
         for (int c = 0; c < chunks; ++c) {
-            const int st = c % kHpStages;
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.full[st], (c / kHpStages) & 1))) {
+            const int st = c % stages;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (c / stages) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t xd = xdesc0 + (uint64_t)(st * (kHpXBytes >> 4));
-                const uint64_t wd = wdesc0 + (uint64_t)(st * ((NT / 64) * kHpWBox >> 4));
+                const uint64_t wd = wdesc0 + (uint64_t)(st * (Lay::kWStage >> 4));
 #pragma unroll
                 for (int k16 = 0; k16 < kHpChunk / 16; ++k16)
                     umma_ss(tacc, xd + (uint64_t)(k16 * 2), wd + (uint64_t)(k16 * 128), idesc, (c | k16) ? 1u : 0u);
-                umma_commit(&S.empty[st]);
+                umma_commit(&empty[st]);
             }
             __syncwarp();
         }
         if (lane == 0)
-            umma_commit(&S.done);
+            umma_commit(done);
         __syncwarp();
         if (!ok && lane == 0 && err)
             atomicOr(err, KVATTN_DEVERR_WAIT_TIMEOUT);
     }
 
     // epilogue: row m0 + threadIdx.x, NT columns from TMEM
-    const bool have = __all_sync(0xffffffffu, mbar_wait(&S.done, 0));
+    const bool have = __all_sync(0xffffffffu, mbar_wait(done, 0));
     tc_fence_after();
     const int row = m0 + threadIdx.x;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
@@ -287,13 +295,15 @@ template <int NT>
 cudaError_t launch_head_proj(const CUtensorMap &xm, const CUtensorMap &wm, void *y, int out_fp32, int rows, int heads,
                              int k, int n, int32_t *err, cudaStream_t st)
 {
-    const size_t smem = sizeof(HpSmem<NT>);
+    const int chunks = k / kHpChunk;
+    const int stages = chunks < kHpStages ? chunks : kHpStages;
+    const size_t smem = HpLayout<NT>::bytes(stages);
     cudaError_t e =
         cudaFuncSetAttribute(head_proj_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     const dim3 grid(heads, n / NT, (rows + 127) / 128);
-    head_proj_kernel<NT><<<grid, kHpThreads, smem, st>>>(xm, wm, y, out_fp32, rows, heads, k, n, err);
+    head_proj_kernel<NT><<<grid, kHpThreads, smem, st>>>(xm, wm, y, out_fp32, rows, heads, k, n, stages, err);
     return cudaGetLastError();
 }
 
@@ -399,10 +409,19 @@ extern "C" int kvattn_head_proj(const void *x, const void *w, void *y, int32_t o
     }
     const int fp32 = out_dtype == KVATTN_OUT_FP32;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the widest output tile that still gives about 1.5 CTAs per SM (the
+    // work is a stream of W; narrow tiles re-read x, wide tiles leave SMs idle)
+    const long long per_tile = (long long)heads * ((rows + 127) / 128);
+    const long long want = 3LL * sm_count() / 2;
+    int nt = 64;
+    if (n % 256 == 0 && per_tile * (n / 256) >= want)
+        nt = 256;
+    else if (n % 128 == 0 && per_tile * (n / 128) >= want)
+        nt = 128;
     cudaError_t e;
-    if (n % 256 == 0)
+    if (nt == 256)
         e = launch_head_proj<256>(xm, wm, y, fp32, rows, heads, k, n, device_error, s);
-    else if (n % 128 == 0)
+    else if (nt == 128)
         e = launch_head_proj<128>(xm, wm, y, fp32, rows, heads, k, n, device_error, s);
     else
         e = launch_head_proj<64>(xm, wm, y, fp32, rows, heads, k, n, device_error, s);
