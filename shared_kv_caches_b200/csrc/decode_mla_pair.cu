@@ -57,6 +57,8 @@
 // arrival can reach a CTA that has left.
 #include <math.h>
 
+#include <type_traits>
+
 #include "latent_common.cuh"
 
 namespace kvattn {
@@ -236,19 +238,6 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kThreads, 1)
         const uint64_t qdesc0 = smem_desc(smem_u32(&S.q[0][0]), 16, 1024, 2);
         // the partner's P: K-major, 64-byte rows, 64-byte swizzle (8-row atoms of 512 bytes)
         const uint64_t pdesc0 = smem_desc(smem_u32(S.pp[0]), 16, 512, 4);
-        // key box kb (this CTA's 32 token rows): from V (own half, rows
-        // 32r..) or E (partner's half, rope); offset within its ring slot in
-        // 16-byte units
-        bool kin_v[kNKB];
-        uint32_t koff[kNKB];
-#pragma unroll
-        for (int kb = 0; kb < kNKB; ++kb) {
-            kin_v[kb] = kb < kNKB - 1 && kb / kNVB == r;
-            const uint32_t off = kb == kNKB - 1 ? kNVB * kEBoxBytes
-                                 : kin_v[kb]   ? (kb % kNVB) * kVBoxBytes + r * kEBoxBytes
-                                               : (kb % kNVB) * kEBoxBytes;
-            koff[kb] = off >> 4;
-        }
         // zero value rows [ntok, 64) of V slot vs (whole 128-byte rows, so
         // the swizzle does not matter); the rows also hold the own-half key
         // rows past the context, whose scores the softmax masks anyway
@@ -265,24 +254,37 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
         };
+        // the score MMAs of page j, in one fully unrolled copy per rank: the
+        // box sources and offsets are constants, so each MMA issues with no
+        // address work (the issuing thread otherwise sets the pace)
+        auto issue_s_rank = [&](auto rank, int j) {
+            constexpr int R = decltype(rank)::value;
+            const uint32_t d = tS + (j & 1) * kHalfTok;
+            const uint64_t ed = edesc0 + (uint64_t)((j % kEStages) * (kEBytes >> 4));
+            const uint64_t vd = kvdesc0 + (uint64_t)((j % kVStages) * (kVBytes >> 4));
+#pragma unroll
+            for (int kb = 0; kb < kNKB; ++kb) {
+                const bool in_v = kb < kNKB - 1 && kb / kNVB == R;
+                const uint32_t off = (kb == kNKB - 1 ? kNVB * kEBoxBytes
+                                      : in_v       ? (kb % kNVB) * kVBoxBytes + R * kEBoxBytes
+                                                   : (kb % kNVB) * kEBoxBytes) >> 4;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t bd = (in_v ? vd : ed) + (uint64_t)(off + k * 2);
+                    const uint32_t acc = (kb | k) ? 1u : 0u;
+                    if (kb < kNQT)
+                        umma_ts(d, tQ + kb * 32 + k * 8, bd, kIdescS, acc);
+                    else
+                        umma_ss(d, qdesc0 + (uint64_t)((kb - kNQT) * (kQChunkBytes >> 4) + k * 2), bd, kIdescS, acc);
+                }
+            }
+        };
         auto issue_s = [&](int j) {
             if (lane == 0) {
-                const uint32_t d = tS + (j & 1) * kHalfTok;
-                const uint64_t ed = edesc0 + (uint64_t)((j % kEStages) * (kEBytes >> 4));
-                const uint64_t vd = kvdesc0 + (uint64_t)((j % kVStages) * (kVBytes >> 4));
-#pragma unroll
-                for (int kb = 0; kb < kNKB; ++kb) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = (kin_v[kb] ? vd : ed) + (uint64_t)(koff[kb] + k * 2);
-                        const uint32_t acc = (kb | k) ? 1u : 0u;
-                        if (kb < kNQT)
-                            umma_ts(d, tQ + kb * 32 + k * 8, bd, kIdescS, acc);
-                        else
-                            umma_ss(d, qdesc0 + (uint64_t)((kb - kNQT) * (kQChunkBytes >> 4) + k * 2), bd, kIdescS,
-                                    acc);
-                    }
-                }
+                if (r == 0)
+                    issue_s_rank(std::integral_constant<int, 0>{}, j);
+                else
+                    issue_s_rank(std::integral_constant<int, 1>{}, j);
                 umma_commit(&S.s_full[j & 1]);
                 umma_commit(&S.e_empty[j % kEStages]);
             }
