@@ -20,6 +20,10 @@
  *   latent head serves one group of query heads.
  *   MLRA page, the GQA and MQA bullets: a group of query heads (or all of
  *   them) shares one K/V head.
+ *   GTA/GLA page (jsbsmhs.com/zixun/902167), "Grouped Tied Attention": the
+ *   heads of a group share one key-value state, tied: the cached vector is
+ *   both the key and the value (MFA page, jsqmd.com/news/79551: key reuse,
+ *   MFA-KR, read as the same tie on MFA's single wide head).
  *
  * Readings where the pages are silent:
  *   - the 1/sqrt(d) factor is the caller's sm_scale and multiplies the whole
@@ -29,7 +33,8 @@
  *   - MLRA keeps one lse per (head, branch) and sums the normalised branch
  *     outputs in latent space;
  *   - GLA: head h belongs to group h / (H / G); the RoPE key is shared by all
- *     groups; MLRA: every head attends every branch with its own query slice.
+ *     groups; MLRA: every head attends every branch with its own query slice;
+ *   - GTA: head h uses tied state h / (H / G), no separate rope part.
  *
  * Per (sequence b, head h[, branch r]) the softmax is taken the plain way, in
  * two passes over the scores: s_j for every cached token, m = max_j s_j,
@@ -40,7 +45,8 @@
  *
  * Cache layouts: latent pool [num_pages][page_size][num_kv*d_nope + d_rope],
  * row = [c_0 | ... | c_{num_kv-1} | k_rope]; GQA/MQA pool
- * [num_pages][2 (K,V)][page_size][num_kv][d_nope].  Token j of sequence b is
+ * [num_pages][2 (K,V)][page_size][num_kv][d_nope]; GTA pool (one tied plane)
+ * [num_pages][page_size][num_kv][d_nope].  Token j of sequence b is
  * slot j % page_size of page block_table[b][j / page_size] (contiguous mode:
  * page b*max_pages_per_seq + j / page_size).
  */
@@ -50,7 +56,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_GQA = 0, ORC_MQA = 1, ORC_MLA = 2, ORC_GLA = 3, ORC_MLRA = 4 };
+enum { ORC_GQA = 0, ORC_MQA = 1, ORC_MLA = 2, ORC_GLA = 3, ORC_MLRA = 4, ORC_GTA = 5 };
 enum { ORC_BF16 = 0, ORC_F64 = 1 };
 
 typedef struct {
@@ -86,6 +92,9 @@ static double elem(const void *base, int type, size_t i)
 
 static int is_latent(int v) { return v == ORC_MLA || v == ORC_GLA || v == ORC_MLRA; }
 
+/* Planes of a GQA/MQA page: K and V, or one tied plane (GTA). */
+static size_t planes(const orc_shape *s) { return s->variant == ORC_GTA ? 1 : 2; }
+
 /* Physical page of the i-th logical page of sequence b. */
 static int64_t page_of(const orc_job *J, int b, int i)
 {
@@ -107,7 +116,7 @@ static size_t key_index(const orc_shape *s, int64_t page, int slot, int u, int d
             return base + (size_t)u * dn + d;
         return base + (size_t)s->num_kv * dn + (d - dn);
     }
-    return (((size_t)page * 2 + 0) * s->page_size + slot) * s->num_kv * dn + (size_t)u * dn + d;
+    return (((size_t)page * planes(s) + 0) * s->page_size + slot) * s->num_kv * dn + (size_t)u * dn + d;
 }
 
 /* Element offset of value element d of token slot (page, slot), unit u. */
@@ -118,7 +127,8 @@ static size_t value_index(const orc_shape *s, int64_t page, int slot, int u, int
         size_t row = (size_t)s->num_kv * dn + (size_t)s->d_rope;
         return ((size_t)page * s->page_size + slot) * row + (size_t)u * dn + d;
     }
-    return (((size_t)page * 2 + 1) * s->page_size + slot) * s->num_kv * dn + (size_t)u * dn + d;
+    /* the V plane; a tied pool has one plane, its vector is the value too */
+    return (((size_t)page * planes(s) + planes(s) - 1) * s->page_size + slot) * s->num_kv * dn + (size_t)u * dn + d;
 }
 
 /* Attention of one query row against all cached tokens of sequence b through
@@ -256,7 +266,7 @@ int orc_decode(const orc_shape *s, int32_t elem_type, const void *q_nope, const 
                double sm_scale, const int32_t *b_list, int32_t n_b, const int32_t *h_list,
                int32_t n_h, double *out, double *lse, int32_t nthreads, int32_t branch_out)
 {
-    if (!s || s->variant < 0 || s->variant > 4 || s->num_kv <= 0 || s->num_q_heads <= 0 ||
+    if (!s || s->variant < 0 || s->variant > ORC_GTA || s->num_kv <= 0 || s->num_q_heads <= 0 ||
         s->d_nope <= 0 || s->d_rope < 0 || s->page_size <= 0)
         return -3;
     if (s->variant != ORC_MLA && s->variant != ORC_MLRA && s->num_q_heads % s->num_kv)

@@ -24,7 +24,7 @@ _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-VARIANT_IDS = {"gqa": 0, "mqa": 1, "mla": 2, "gla": 3, "mlra": 4}
+VARIANT_IDS = {"gqa": 0, "mqa": 1, "mla": 2, "gla": 3, "mlra": 4, "gta": 5}
 
 
 class _Shape(ctypes.Structure):

@@ -21,7 +21,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 MUTATIONS = {
     "drop_rope": ("q[dn + d] = elem(J->q_rope, J->elem_type, q_row * dr + d);", "q[dn + d] = 0.0;"),
     "sign": ("Z += exp(sc[j] - m);", "Z += exp(m - sc[j]);"),
-    "v_from_k_plane": ("return (((size_t)page * 2 + 1)", "return (((size_t)page * 2 + 0)"),
+    "v_from_k_plane": ("return (((size_t)page * planes(s) + planes(s) - 1)", "return (((size_t)page * planes(s) + 0)"),
     "gla_group": ("u = h / (H / s->num_kv);", "u = h % s->num_kv;"),
     "mlra_q_index": ("size_t q_row = ((size_t)b * H + h) * R + r;",
                      "size_t q_row = ((size_t)b * R + r) * H + h;"),

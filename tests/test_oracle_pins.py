@@ -40,6 +40,8 @@ def _tiny_f64(variant, B=2, H=4, NU=2, dn=6, dr=3, lens=(5, 3), ps=2, seed=0):
     num_pages = sum(need) + 2
     if latent:
         kv = rng.standard_normal((num_pages, ps, NU * dn + dr))
+    elif variant == "gta":
+        kv = rng.standard_normal((num_pages, ps, NU, dn))
     else:
         kv = rng.standard_normal((num_pages, 2, ps, NU, dn))
     perm = rng.permutation(num_pages)
@@ -310,6 +312,37 @@ def test_gla_is_two_mla_problems(oracle_mod):
         o, l = _run(oracle_mod, Q, 0.7)
         np.testing.assert_allclose(out[:, hs], o, rtol=0, atol=1e-14)
         np.testing.assert_allclose(lse[:, hs], l, rtol=0, atol=1e-14)
+
+
+def test_gta_is_gqa_with_keys_and_values_tied(oracle_mod):
+    """GTA/GLA page, "Grouped Tied Attention": the cached vector of a group is
+    both key and value.  GTA on a one-plane pool = GQA on the pool whose K and
+    V planes are both that plane; with one group (MFA page, key reuse) it is
+    MQA on such a pool."""
+    P = _tiny_f64("gta", H=6, NU=3, seed=63)
+    out, lse = _run(oracle_mod, P, 0.45)
+    both = np.stack([P["kv"], P["kv"]], axis=1)          # [pages][2][ps][NU][d]
+    out_g, lse_g = _run(oracle_mod, dict(P, variant="gqa", kv=both), 0.45)
+    np.testing.assert_array_equal(out, out_g)
+    np.testing.assert_array_equal(lse, lse_g)
+    M = _tiny_f64("gta", H=5, NU=1, seed=64)
+    out_m, _ = _run(oracle_mod, M, 0.45)
+    out_q, _ = _run(oracle_mod, dict(M, variant="mqa", kv=np.stack([M["kv"], M["kv"]], axis=1)), 0.45)
+    np.testing.assert_array_equal(out_m, out_q)
+
+
+def test_gta_brute_force_tiny(oracle_mod):
+    """Brute force through numpy: softmax(scale q K^T) K with the group's tied
+    vectors gathered by fancy indexing."""
+    P = _tiny_f64("gta", H=4, NU=2, seed=65)
+    out, lse = _run(oracle_mod, P, 0.41)
+    for b in range(P["B"]):
+        pages, slots = _gather_rows(P, b)
+        for h in range(P["H"]):
+            KV = P["kv"][pages, slots, h // (P["H"] // P["NU"])]
+            o, l = _softmax_attend(P["qn"][b, h], KV, KV, 0.41)
+            np.testing.assert_allclose(out[b, h], o, rtol=1e-12, atol=1e-13)
+            assert abs(lse[b, h] - l) < 1e-12
 
 
 def test_gqa_is_mha_with_repeated_kv(oracle_mod):
