@@ -11,7 +11,8 @@ at the DeepSeek-V3 shape (batch 64, 128 query heads, latent 512 + rope 64,
 ragged contexts drawn uniformly from [4096, 32768] on a paged 64-token bf16
 cache with a permuted block table), the largest problem that fits one GPU;
 ``suite`` carries the same figures for GQA, MFA, GLA-2 and the four MLRA-4
-shapes.  ``--workload NAME`` times one problem (or ``gqa+mfa``, the GQA and
+shapes, and GTA and MFA-KR (the GQA and MFA shapes with tied keys and
+values).  ``--workload NAME`` times one problem (or ``gqa+mfa``, the GQA and
 MFA layers together as one step); ``--workload steps`` only the steps either
 side of attention.
 
@@ -58,7 +59,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOAD_SETS = {"gqa+mfa": ("gqa", "mfa")}
-SUITE = ("mla", "gqa", "mfa", "gla", "mlra_128k", "mlra_512k", "mlra_1m", "mlra_b8_128k")
+SUITE = ("mla", "gqa", "mfa", "gla", "mlra_128k", "mlra_512k", "mlra_1m", "mlra_b8_128k", "gta", "mfa_kr")
 DEFAULT_WORKLOAD = "suite"
 METRIC = "decode_attn_tokens_per_s"
 UNIT = "tokens/s"

@@ -27,6 +27,10 @@
  *   KVATTN_MLRA num_kv = R branches of d_nope each plus one shared rope key;
  *               every head attends every branch with its own query slice and
  *               the R normalised branch outputs are summed (latent space)
+ *   KVATTN_GTA  num_kv tied states of d_nope: the cached vector of group g is
+ *               both key and value for heads g*H/G .. (GTA/GLA page, "Grouped
+ *               Tied Attention"); num_kv = 1 with one wide head is the MFA
+ *               page's key reuse (MFA-KR)
  *
  * Memory (all device pointers, row-major, caller-owned):
  *   q_nope     bf16 [B][Q][H][d_nope]        (MLRA [B][Q][H][R][d_nope]), Q = q_len
@@ -34,7 +38,8 @@
  *              d_rope == 0 (GQA/MQA)
  *   kv_cache   latent variants: bf16 [num_pages][page_size][num_kv*d_nope + d_rope],
  *              each token row [c_0 | ... | c_{num_kv-1} | k_rope];
- *              GQA/MQA: bf16 [num_pages][2 (K, V)][page_size][num_kv][d_nope]
+ *              GQA/MQA: bf16 [num_pages][2 (K, V)][page_size][num_kv][d_nope];
+ *              GTA: bf16 [num_pages][page_size][num_kv][d_nope] (one tied plane)
  *   block_table int32 [B][max_pages_per_seq]: physical page of each logical
  *              64-token page; NULL = contiguous cache, sequence b owns pages
  *              b*max_pages_per_seq .. b*max_pages_per_seq + max_pages_per_seq-1
@@ -80,7 +85,8 @@ enum kvattn_variant {
     KVATTN_MQA = 1,
     KVATTN_MLA = 2,
     KVATTN_GLA = 3,
-    KVATTN_MLRA = 4
+    KVATTN_MLRA = 4,
+    KVATTN_GTA = 5
 };
 
 enum kvattn_out_dtype { KVATTN_OUT_BF16 = 0, KVATTN_OUT_FP32 = 1 };
@@ -297,7 +303,9 @@ int kvattn_rope(void *x, int32_t rows, int32_t row_elems, int32_t rot_offset, in
  * fields are checked as for decode).  new_kv, bf16, caller-owned:
  *   latent variants  [B][Q][num_kv*d_nope + d_rope], [c_0 | ... | k^R] with
  *                    k^R not yet rotated;
- *   GQA/MQA          [B][Q][2][num_kv][d_nope], K then V.
+ *   GQA/MQA          [B][Q][2][num_kv][d_nope], K then V;
+ *   GTA              [B][Q][num_kv][d_nope], the tied vectors (stored as
+ *                    given: rope_base must be 0).
  * pos int32 [B][Q]: the cache position of each token (slot pos % 64 of page
  * block_table[b][pos / 64]; block_table NULL = contiguous, as in decode).
  * rope_base > 1 rotates k^R (latent) or every K head (GQA/MQA) at its

@@ -20,8 +20,8 @@ L2_BYTES = 126 * 1024 * 1024
 
 def kv_bytes_per_token(shape) -> int:
     """Cache bytes one context token contributes (the whole row is read once:
-    latent row, or K and V of every KV head)."""
-    if shape.latent:
+    latent row, the tied vectors of GTA, or K and V of every KV head)."""
+    if shape.latent or shape.tied:
         return 2 * shape.row_elems
     return 2 * 2 * shape.num_kv * shape.d_nope
 

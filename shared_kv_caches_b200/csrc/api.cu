@@ -20,7 +20,7 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
 {
     if (!p || !pr)
         return KVATTN_ERR_INVALID_ARG;
-    if (variant < KVATTN_GQA || variant > KVATTN_MLRA)
+    if (variant < KVATTN_GQA || variant > KVATTN_GTA)
         return KVATTN_ERR_UNSUPPORTED;
     if (p->batch < 1 || p->num_q_heads < 1 || p->num_kv < 1 || p->d_nope < 1 || p->d_rope < 0 ||
         p->max_pages_per_seq < 1 || p->num_pages < 1 || p->max_seq_len < 0 || p->num_splits < 0)
@@ -47,7 +47,7 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
         return KVATTN_ERR_INVALID_ARG;
     if ((variant == KVATTN_MQA || variant == KVATTN_MLA) && p->num_kv != 1)
         return KVATTN_ERR_INVALID_ARG;
-    if ((variant == KVATTN_GQA || variant == KVATTN_GLA) && p->num_q_heads % p->num_kv)
+    if ((variant == KVATTN_GQA || variant == KVATTN_GLA || variant == KVATTN_GTA) && p->num_q_heads % p->num_kv)
         return KVATTN_ERR_INVALID_ARG;
     if (variant == KVATTN_MLRA && p->num_kv > 16)
         return KVATTN_ERR_UNSUPPORTED;
@@ -76,6 +76,7 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
     pr->out_dtype = p->out_dtype;
     pr->paged = true;
     pr->branch_out = p->branch_out != 0;
+    pr->kv_planes = variant == KVATTN_GTA ? 1 : 2;
     return KVATTN_OK;
 }
 
@@ -341,6 +342,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     a.dn = pr.dn;
     a.dr = pr.dr;
     a.row = pr.row;
+    a.kv_planes = pr.kv_planes;
     a.HPU = pr.HPU;
     a.HU = pr.HU;
     a.mpps = pr.mpps;

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads) generic_decode_kernel(const DecodeAr
                 const __nv_bfloat16 *row = a.kv + ((size_t)page * kPage + t) * a.row;
                 src = v * 8 < a.dn ? row + (size_t)u * a.dn + v * 8 : row + (size_t)a.NU * a.dn + (v * 8 - a.dn);
             } else {
-                src = a.kv + (((size_t)page * 2 + 0) * kPage + t) * a.row + (size_t)u * a.dn + v * 8;
+                src = a.kv + (((size_t)page * a.kv_planes + 0) * kPage + t) * a.row + (size_t)u * a.dn + v * 8;
             }
             const uint4 w = *reinterpret_cast<const uint4 *>(src);
             uint32_t *dst = ks + (t * KS) / 2 + v * 4;
@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads) generic_decode_kernel(const DecodeAr
             for (int idx = tid; idx < ntok * vec_v; idx += kThreads) {
                 const int t = idx / vec_v, v = idx % vec_v;
                 const __nv_bfloat16 *src =
-                    a.kv + (((size_t)page * 2 + 1) * kPage + t) * a.row + (size_t)u * a.dn + v * 8;
+                    a.kv + (((size_t)page * a.kv_planes + a.kv_planes - 1) * kPage + t) * a.row + (size_t)u * a.dn +
+                    v * 8;
                 const uint4 w = *reinterpret_cast<const uint4 *>(src);
                 uint32_t *dst = vs + (t * VS) / 2 + v * 4;
                 dst[0] = w.x;

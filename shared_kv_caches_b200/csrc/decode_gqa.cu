@@ -138,13 +138,17 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
                     continue;
                 }
                 S.skip[st] = 0;
-                mbar_arrive_expect_tx(&S.full[st], STAGE_BYTES);
-                const int zk = (int)(page * 2 * kPage), zv = zk + kPage;
+                // tied keys and values (GTA): one tile serves as both
+                const bool tied = a.kv_planes == 1;
+                mbar_arrive_expect_tx(&S.full[st], tied ? TILE_BYTES : STAGE_BYTES);
+                const int zk = (int)(page * a.kv_planes * kPage), zv = zk + kPage;
                 unsigned char *t = S.tiles[st];
                 tma_load_3d(t, &kv_map, 0, kvh, zk, &S.full[st]);
                 tma_load_3d(t + BOX_BYTES, &kv_map, 64, kvh, zk, &S.full[st]);
-                tma_load_3d(t + TILE_BYTES, &kv_map, 0, kvh, zv, &S.full[st]);
-                tma_load_3d(t + TILE_BYTES + BOX_BYTES, &kv_map, 64, kvh, zv, &S.full[st]);
+                if (!tied) {
+                    tma_load_3d(t + TILE_BYTES, &kv_map, 0, kvh, zv, &S.full[st]);
+                    tma_load_3d(t + TILE_BYTES + BOX_BYTES, &kv_map, 64, kvh, zv, &S.full[st]);
+                }
             }
         }
         return;
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
         const int nw = S.skip[st] ? 0 : min(max(ntok - t0, 0), TPW);
         if (nw > 0) {
             unsigned char *Kb = S.tiles[st];
-            unsigned char *Vb = Kb + TILE_BYTES;
+            unsigned char *Vb = a.kv_planes == 1 ? Kb : Kb + TILE_BYTES;
             if (nw < TPW) {
                 // value rows of this warp past the context: 0 * NaN would poison the MMA
                 for (int idx = lane; idx < (TPW - nw) * (D / 8); idx += 32)
@@ -317,7 +321,7 @@ bool gqa_supported(const Problem &pr)
 cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st)
 {
     CUtensorMap map;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.NU, (cuuint64_t)a.num_pages * 2 * kPage};
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.NU, (cuuint64_t)a.num_pages * a.kv_planes * kPage};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.NU * D * 2};
     const cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
     if (encode_tiled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.kv), dims, strides,

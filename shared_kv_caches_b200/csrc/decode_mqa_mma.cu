@@ -121,13 +121,16 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
                     continue;
                 }
                 S.skip[st] = 0;
-                mbar_arrive_expect_tx(&S.full[st], STAGE_BYTES);
-                const int zk = (int)(page * 2 * kPage), zv = zk + kPage;
+                // tied keys and values (MFA-KR): one tile serves as both
+                const bool tied = a.kv_planes == 1;
+                mbar_arrive_expect_tx(&S.full[st], tied ? TILE_BYTES : STAGE_BYTES);
+                const int zk = (int)(page * a.kv_planes * kPage), zv = zk + kPage;
                 unsigned char *t = S.tiles[st];
 #pragma unroll
                 for (int x = 0; x < D / 64; ++x) {
                     tma_load_3d(t + x * BOX_BYTES, &kv_map, 64 * x, kvh, zk, &S.full[st]);
-                    tma_load_3d(t + TILE_BYTES + x * BOX_BYTES, &kv_map, 64 * x, kvh, zv, &S.full[st]);
+                    if (!tied)
+                        tma_load_3d(t + TILE_BYTES + x * BOX_BYTES, &kv_map, 64 * x, kvh, zv, &S.full[st]);
                 }
             }
         }
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, 1) mqa_mma_decode_kernel(const __grid
         }
         const int ntok = S.skip[st] ? 0 : min(kPage, L - (p0 + i) * kPage);
         unsigned char *Kb = S.tiles[st];
-        unsigned char *Vb = Kb + TILE_BYTES;
+        unsigned char *Vb = a.kv_planes == 1 ? Kb : Kb + TILE_BYTES;
         if (ntok > 0 && ntok < kPage) {
             // zero this warp's value slice of the slots past the context (the two
             // warps of a value half write the same zeros, then both wait)
@@ -289,7 +292,7 @@ bool mqa_mma_supported(const Problem &pr)
 cudaError_t launch_mqa_mma(const DecodeArgs &a, cudaStream_t st)
 {
     CUtensorMap map;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.NU, (cuuint64_t)a.num_pages * 2 * kPage};
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.NU, (cuuint64_t)a.num_pages * a.kv_planes * kPage};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.NU * D * 2};
     const cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
     if (encode_tiled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.kv), dims, strides,

@@ -29,6 +29,7 @@ struct Problem {
     int mpps, num_pages, max_seq_len, out_dtype;
     bool latent, mlra, paged;
     bool branch_out;   // MLRA: the R branch outputs side by side instead of their sum
+    int kv_planes;     // GQA/MQA pages: 2 (K, V); GTA: 1 (the tied vector is key and value)
 };
 
 // Arguments of every decode kernel.  Partial results go to the workspace as
@@ -51,6 +52,7 @@ struct DecodeArgs {
     int num_splits, pages_per_split, head_chunks;
     int latent, mlra;
     int q_len;                    // query tokens per sequence; B counts (sequence, position) rows
+    int kv_planes;                // GQA/MQA pages: 2 (K, V); GTA: 1 (keys are the values)
     float scale_log2;             // sm_scale * log2(e): scores kept in base 2
 };
 

@@ -365,6 +365,15 @@ extern "C" int kvattn_append_kv(int32_t variant, const kvattn_params *p, const v
         a.copy = pr.NU * pr.dn;
         a.rot_width = pr.dr;
         a.rot_count = (rope_base > 0.f && pr.dr > 0) ? 1 : 0;
+    } else if (pr.kv_planes == 1) {
+        // tied keys and values (GTA, MFA-KR): the row is the value too, so it
+        // is stored as given (the pages do not place RoPE for the tie)
+        if (rope_base != 0.f)
+            return KVATTN_ERR_INVALID_ARG;
+        a.planes = 1;
+        a.copy = pr.row;
+        a.rot_width = 0;
+        a.rot_count = 0;
     } else {
         a.planes = 2;
         a.copy = 0;

@@ -18,9 +18,9 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvattn.so")
 
-KVATTN_GQA, KVATTN_MQA, KVATTN_MLA, KVATTN_GLA, KVATTN_MLRA = range(5)
+KVATTN_GQA, KVATTN_MQA, KVATTN_MLA, KVATTN_GLA, KVATTN_MLRA, KVATTN_GTA = range(6)
 VARIANTS = {"gqa": KVATTN_GQA, "mqa": KVATTN_MQA, "mla": KVATTN_MLA, "gla": KVATTN_GLA,
-            "mlra": KVATTN_MLRA}
+            "mlra": KVATTN_MLRA, "gta": KVATTN_GTA}
 KVATTN_OUT_BF16, KVATTN_OUT_FP32 = 0, 1
 KVATTN_OK = 0
 KVATTN_ERR_INVALID_ARG = -1

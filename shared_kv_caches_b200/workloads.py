@@ -35,7 +35,7 @@ import math
 
 import numpy as np
 
-VARIANT_IDS = {"gqa": 0, "mqa": 1, "mla": 2, "gla": 3, "mlra": 4}
+VARIANT_IDS = {"gqa": 0, "mqa": 1, "mla": 2, "gla": 3, "mlra": 4, "gta": 5}
 LATENT_VARIANTS = ("mla", "gla", "mlra")
 
 BF16_NAN = 0x7FC0
@@ -97,8 +97,13 @@ class Shape:
         return self.num_kv * self.d_nope
 
     @property
+    def tied(self) -> bool:
+        """GTA / MFA-KR: one cached vector per unit is both key and value."""
+        return self.variant == "gta"
+
+    @property
     def page_elems(self) -> int:
-        if self.latent:
+        if self.latent or self.tied:
             return self.page_size * self.row_elems
         return 2 * self.page_size * self.row_elems
 
@@ -144,6 +149,8 @@ class Shape:
     def pool_shape(self, num_pages: int) -> tuple:
         if self.latent:
             return (num_pages, self.page_size, self.row_elems)
+        if self.tied:
+            return (num_pages, self.page_size, self.num_kv, self.d_nope)
         return (num_pages, 2, self.page_size, self.num_kv, self.d_nope)
 
     def replace(self, **kw) -> "Shape":
@@ -153,7 +160,9 @@ class Shape:
 # The workloads of the decode-attention benchmark suite.  Names state what
 # they are; sizes follow the shapes the pages discuss (DeepSeek-V3-like MLA
 # 512+64, GLA-2 with two 256-wide latent heads, MLRA-4 with four 128-wide
-# branches, GQA 32q/8kv and an MFA-style single wide KV head).
+# branches, GQA 32q/8kv and an MFA-style single wide KV head; GTA and MFA-KR
+# are the same GQA and MFA shapes with keys and values tied into one cached
+# vector).
 WORKLOADS = {
     "tiny_mla": Shape("mla", 2, 8, 1, 64, 16, (512, 512), paged=False, out_dtype="fp32"),
     "gqa": Shape("gqa", 32, 32, 8, 128, 0, (1024, 8192)),
@@ -164,6 +173,8 @@ WORKLOADS = {
     "mlra_512k": Shape("mlra", 1, 128, 4, 128, 64, (524288, 524288)),
     "mlra_1m": Shape("mlra", 1, 128, 4, 128, 64, (1048576, 1048576)),
     "mlra_b8_128k": Shape("mlra", 8, 128, 4, 128, 64, (131072, 131072)),
+    "gta": Shape("gta", 32, 32, 8, 128, 0, (1024, 8192)),
+    "mfa_kr": Shape("gta", 32, 32, 1, 256, 0, (1024, 8192)),
 }
 
 
@@ -267,8 +278,8 @@ def make_inputs(shape: Shape, seed: int = 0, seq_lens=None, poison: bool = True,
             if n == 0 or tail == ps:
                 continue
             page = block_table[b, n - 1] if shape.paged else b * mpps + n - 1
-            if shape.latent:
-                seg = kv[page, tail:, :]
+            if shape.latent or shape.tied:
+                seg = kv[page, tail:]
             else:
                 seg = kv[page, :, tail:, :, :]
             seg[...] = pois(seg.size).reshape(seg.shape)

@@ -82,6 +82,11 @@ SMALL = {
     "mlra1_shard": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=1, ctx=(100, 700)), None),
     "mlra2": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=2, d_nope=256, ctx=(100, 700)), None),
     "mlra8": (W.WORKLOADS["mlra_128k"].replace(batch=2, num_kv=8, d_nope=64, ctx=(100, 700)), None),
+    # tied keys and values: GTA on the GQA kernel, MFA-KR on the MQA kernel,
+    # and a tied shape only the generic kernel covers
+    "gta": (W.WORKLOADS["gta"].replace(batch=3, ctx=(1, 700)), None),
+    "mfa_kr": (W.WORKLOADS["mfa_kr"].replace(batch=3, ctx=(1, 700)), None),
+    "gta_generic": (W.WORKLOADS["gta"].replace(batch=2, num_q_heads=8, num_kv=2, d_nope=64, ctx=(1, 300)), None),
 }
 
 
@@ -102,6 +107,8 @@ SWEEP_SHAPES = {
     "mla": W.WORKLOADS["mla"],
     "gla": W.WORKLOADS["gla"],
     "mlra": W.WORKLOADS["mlra_128k"],
+    "gta": W.WORKLOADS["gta"],
+    "mfa_kr": W.WORKLOADS["mfa_kr"],
 }
 
 
@@ -135,7 +142,7 @@ def _sample(x, shape):
 
 
 @pytest.mark.parametrize("name", ["gqa", "mfa", "mla", "gla", "mlra_128k", "mlra_512k", "mlra_1m",
-                                  "mlra_b8_128k"])
+                                  "mlra_b8_128k", "gta", "mfa_kr"])
 def test_parity_full_size_sampled(dev, oracle_mod, name):
     """Full benchmark sizes, library-chosen launch (as timed by bench.py);
     the oracle computes sampled sequences (and heads for batch 1)."""
@@ -157,6 +164,9 @@ def test_benchmark_shapes_use_the_specialised_kernels(dev):
     for n in ("gla", "mlra_128k", "mlra_1m", "mlra_b8_128k"):
         assert kernel_of(W.WORKLOADS[n]) == "latent_tc", n
     assert kernel_of(W.WORKLOADS["tiny_mla"]) == "generic"
+    assert kernel_of(W.WORKLOADS["gta"]) == "gqa"
+    assert kernel_of(W.WORKLOADS["mfa_kr"]) == "mqa_tc"
+    assert kernel_of(SMALL["gta_generic"][0]) == "generic"
     for name in ("gla1_shard", "gla4", "gla8", "mlra1_shard", "mlra2", "mlra8"):
         assert kernel_of(SMALL[name][0]) == "latent_tc", name
 
@@ -333,6 +343,7 @@ Q_SHAPES = {
     "gla": W.WORKLOADS["gla"].replace(batch=2, ctx=(100, 700)),
     "mlra": W.WORKLOADS["mlra_128k"].replace(batch=2, ctx=(100, 700)),
     "tiny_mla": W.WORKLOADS["tiny_mla"],
+    "gta": W.WORKLOADS["gta"].replace(batch=3, ctx=(1, 700)),
 }
 
 

@@ -163,6 +163,33 @@ def test_append_heads_matches_oracle(dev):
     assert_turned(got[:, 0][touched], ref[:, 0][touched], "append K")
 
 
+def test_append_tied_rows_copies_bits_and_refuses_rope(dev):
+    """GTA / MFA-KR: the tied vector is the value too, so it is stored as given."""
+    import torch
+    from shared_kv_caches_b200 import kvattn as K
+    from shared_kv_caches_b200.device import DeviceProblem
+    s = W.WORKLOADS["gta"].replace(batch=3, ctx=(70, 400), q_len=2)
+    x = W.make_inputs(s, seed=14)
+    rng = np.random.default_rng(15)
+    new = W.f32_to_bf16_bits(rng.standard_normal((s.batch, 2, s.num_kv, s.d_nope)).astype(np.float32))
+    pos = (x["seq_lens"][:, None] - 2 + np.arange(2)).astype(np.int32)
+    p = DeviceProblem(x, dev)
+    before = p.kv.clone()
+    new_d, pos_d = to_dev(new, dev), torch.from_numpy(pos).to(dev)
+    st = K.kvattn_append_kv(p.variant, p.params, new_d.data_ptr(), pos_d.data_ptr(), p.block_table.data_ptr(),
+                            p.kv.data_ptr(), BASE, None, torch.cuda.current_stream(dev).cuda_stream)
+    assert st == K.KVATTN_ERR_INVALID_ARG
+    p.append_kv(new_d, pos_d, 0.0)
+    torch.cuda.synchronize()
+    got = p.kv.cpu().view(torch.int16).numpy().view(np.uint16)
+    ref = before.cpu().view(torch.int16).numpy().view(np.uint16).copy()
+    for b in range(s.batch):
+        for i in range(2):
+            pg, sl = steps.slot_of(x["block_table"], b, int(pos[b, i]), None)
+            ref[pg, sl] = new[b, i]
+    np.testing.assert_array_equal(got, ref)
+
+
 def test_append_without_rope_copies_bits(dev):
     import torch
     from shared_kv_caches_b200.device import DeviceProblem
