@@ -293,20 +293,29 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kThreads, 1)
         // O += [P_0 | P_1] V over the page's 64 tokens (16 per MMA): the
         // tokens of half r come from this CTA's TMEM, the others from the
         // partner's P in shared memory
+        // P.V of page t, one copy per rank: the 16-token steps of this CTA's
+        // half read P from TMEM, the partner's half from shared memory
+        auto issue_pv_rank = [&](auto rank, int t) {
+            constexpr int R = decltype(rank)::value;
+            const uint64_t vd = vdesc0 + (uint64_t)((t % kVStages) * (kVBytes >> 4));
+            const uint32_t pa = tS + (t & 1) * kHalfTok;
+            const uint64_t pd = pdesc0 + (uint64_t)((t & 1) * (kPBytes >> 4));
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
+                if ((s >> 1) == R)
+                    umma_ts(tO, pa + 8 * (s & 1), vd + (uint64_t)(s * 128), kIdescPV, acc);
+                else
+                    umma_ss(tO, pd + (uint64_t)((s & 1) * 2), vd + (uint64_t)(s * 128), kIdescPV, acc);
+            }
+        };
         auto issue_pv = [&](int t) {
             tc_fence_after();
             if (lane == 0) {
-                const uint64_t vd = vdesc0 + (uint64_t)((t % kVStages) * (kVBytes >> 4));
-                const uint32_t pa = tS + (t & 1) * kHalfTok;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
-                    if ((s >> 1) == r)
-                        umma_ts(tO, pa + 8 * (s & 1), vd + (uint64_t)(s * 128), kIdescPV, acc);
-                    else
-                        umma_ss(tO, pdesc0 + (uint64_t)((t & 1) * (kPBytes >> 4) + (s & 1) * 2),
-                                vd + (uint64_t)(s * 128), kIdescPV, acc);
-                }
+                if (r == 0)
+                    issue_pv_rank(std::integral_constant<int, 0>{}, t);
+                else
+                    issue_pv_rank(std::integral_constant<int, 1>{}, t);
                 umma_commit(&S.o_ready);
                 umma_commit(&S.v_empty[t % kVStages]);
                 umma_commit_multicast(&S.pv_done[t & 1], 0x3);
