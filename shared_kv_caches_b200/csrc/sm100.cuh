@@ -70,6 +70,9 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
 // tries (kWaitLimit unless a caller asks for fewer).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = kWaitLimit)
 {
+    // a phase that has already completed is seen by the non-blocking test
+    if (mbar_test(bar, parity))
+        return true;
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity))
             return true;
