@@ -59,7 +59,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOAD_SETS = {"gqa+mfa": ("gqa", "mfa")}
-SUITE = ("mla", "gqa", "mfa", "gla", "mlra_128k", "mlra_512k", "mlra_1m", "mlra_b8_128k", "gta", "mfa_kr")
+SUITE = ("mla", "gqa", "mfa", "gla", "mlra_128k", "mlra_512k", "mlra_1m", "mlra_b8_128k", "gta", "mfa_kr",
+         "gqa_fp8")
 DEFAULT_WORKLOAD = "suite"
 METRIC = "decode_attn_tokens_per_s"
 UNIT = "tokens/s"
@@ -110,12 +111,15 @@ def describe(names):
                       "mlra": f"{s.num_kv} branches x {s.d_nope} + shared rope {s.d_rope}"}[s.variant]
         else:
             kvdesc = f"{s.num_kv} kv heads x {s.d_nope}"
+        if s.cache_dtype != "bf16":
+            kvdesc += f" {s.cache_dtype} e4m3 cache (k_scale {s.k_scale}, v_scale {s.v_scale})"
         parts.append(f"{s.variant} B={s.batch} H={s.num_q_heads} {kvdesc} ctx {ctx}")
     return "; ".join(parts)
 
 
 KERNEL_SOURCES = {
     "gqa": ["decode_gqa.cu"],
+    "gqa_fp8": ["decode_gqa_fp8.cu"],
     "mqa_tc": ["decode_mqa_mma.cu"],
     "latent_tc": ["decode_latent_tc.cu", "latent_common.cuh"],
     "latent_pair": ["decode_mla_pair.cu", "latent_common.cuh"],

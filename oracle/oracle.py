@@ -102,6 +102,39 @@ def _run(variant, batch, num_q_heads, num_kv, d_nope, d_rope, page_size, max_pag
     return out, lse
 
 
+def e4m3_value(codes) -> np.ndarray:
+    """fp8 e4m3 codes -> float64, from the format: sign in bit 7, exponent in
+    bits 6..3 with bias 7, mantissa in bits 2..0; exponent 0 holds subnormals
+    (m / 8 * 2^-6); exponent 15 with mantissa 7 is NaN (there are no
+    infinities)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.power(2.0, e - 7))
+    return sign * np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def _bf16_value(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64 (a bf16 is the top half of an fp32)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def _decode_fp8(inputs: dict, b_list, nthreads, sm_scale, h_list):
+    """GQA over an fp8 cache: the attention of the dequantised cache, key =
+    k_scale * K8 (plane 0), value = v_scale * V8 (plane 1), in fp64."""
+    s = inputs["shape"]
+    kv = e4m3_value(inputs["kv"])
+    kv[:, 0] *= s.k_scale
+    kv[:, 1] *= s.v_scale
+    scale = inputs["sm_scale"] if sm_scale is None else sm_scale
+    return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
+                inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 1,
+                _bf16_value(inputs["q_nope"]), None, kv, inputs["block_table"],
+                inputs["seq_lens"], scale, b_list, nthreads, h_list)
+
+
 def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None, h_list=None,
            branch_out: bool = False):
     """fp64 decode attention of a workload dict (from ``workloads.make_inputs``).
@@ -116,6 +149,8 @@ def decode(inputs: dict, b_list=None, nthreads: int | None = None, sm_scale=None
     s = inputs["shape"]
     if getattr(s, "q_len", 1) > 1:
         return decode_queries(inputs, b_list, nthreads, sm_scale, h_list, branch_out)
+    if getattr(s, "cache_dtype", "bf16") == "fp8":
+        return _decode_fp8(inputs, b_list, nthreads, sm_scale, h_list)
     scale = inputs["sm_scale"] if sm_scale is None else sm_scale
     return _run(s.variant, s.batch, s.num_q_heads, s.num_kv, s.d_nope, s.d_rope, s.page_size,
                 inputs["max_pages_per_seq"], inputs["num_pages"], s.paged, 0,

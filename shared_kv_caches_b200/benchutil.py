@@ -23,7 +23,8 @@ def kv_bytes_per_token(shape) -> int:
     latent row, the tied vectors of GTA, or K and V of every KV head)."""
     if shape.latent or shape.tied:
         return 2 * shape.row_elems
-    return 2 * 2 * shape.num_kv * shape.d_nope
+    elem = 1 if getattr(shape, "cache_dtype", "bf16") == "fp8" else 2
+    return elem * 2 * shape.num_kv * shape.d_nope
 
 
 def flops_per_token(shape) -> int:

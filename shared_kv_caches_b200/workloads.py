@@ -42,6 +42,8 @@ BF16_NAN = 0x7FC0
 BF16_POS_1E4 = 0x461C
 BF16_NEG_1E4 = 0xC61C
 POISON_BITS = np.array([BF16_NAN, BF16_POS_1E4, BF16_NEG_1E4], dtype=np.uint16)
+# fp8 (e4m3) poison: NaN, +448 and -448 (the largest magnitudes)
+POISON_FP8 = np.array([0x7F, 0x7E, 0xFE], dtype=np.uint8)
 
 _CHUNK = 1 << 24
 
@@ -72,6 +74,9 @@ class Shape:
     input_scale: float = 1.0
     q_len: int = 1          # query tokens per sequence (the newest q_len cached tokens)
     branch_out: bool = False  # MLRA: the branch outputs side by side instead of their sum
+    cache_dtype: str = "bf16"  # "fp8": the cache holds e4m3 bytes (GQA), key = k_scale * K8, value = v_scale * V8
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
     @property
     def variant_id(self) -> int:
@@ -175,6 +180,7 @@ WORKLOADS = {
     "mlra_b8_128k": Shape("mlra", 8, 128, 4, 128, 64, (131072, 131072)),
     "gta": Shape("gta", 32, 32, 8, 128, 0, (1024, 8192)),
     "mfa_kr": Shape("gta", 32, 32, 1, 256, 0, (1024, 8192)),
+    "gqa_fp8": Shape("gqa", 32, 32, 8, 128, 0, (1024, 8192), cache_dtype="fp8", k_scale=0.5, v_scale=2.0),
 }
 
 
@@ -204,6 +210,39 @@ def _normal_bf16(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
         if scale != 1.0:
             draw *= np.float32(scale)
         out[start:stop] = f32_to_bf16_bits(draw)
+    return out.reshape(shape)
+
+
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """float values -> fp8 e4m3 codes (sign, 4 exponent bits with bias 7, 3
+    mantissa bits), rounded to nearest even and saturated at +-448; NaN maps
+    to 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.where(np.signbit(x), 0x80, 0).astype(np.int64)
+    nan = np.isnan(x)
+    a = np.where(nan, 0.0, np.minimum(np.abs(x), 448.0))
+    m, e = np.frexp(a)                                   # a = m 2^e, 0.5 <= m < 1
+    exp = e.astype(np.int64) - 1                         # a = (2m) 2^exp
+    normal = (exp >= -6) & (a > 0)
+    # normal: code = (exp + 7) * 8 + rint((2m - 1) * 8); a mantissa carry moves to the next exponent
+    code_n = (exp + 7) * 8 + np.rint((2.0 * m - 1.0) * 8.0).astype(np.int64)
+    # subnormal (and the smallest normal reached by rounding up): multiples of 2^-9
+    code_s = np.rint(np.ldexp(a, 9)).astype(np.int64)
+    code = np.where(normal, code_n, code_s)
+    code = np.minimum(code, 0x7E)
+    out = (code | sign).astype(np.uint8)
+    return np.where(nan, np.uint8(0x7F), out)
+
+
+def _normal_e4m3(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = np.empty(n, dtype=np.uint8)
+    for start in range(0, n, _CHUNK):
+        stop = min(n, start + _CHUNK)
+        draw = rng.standard_normal(stop - start, dtype=np.float32)
+        if scale != 1.0:
+            draw *= np.float32(scale)
+        out[start:stop] = f32_to_e4m3_bits(draw)
     return out.reshape(shape)
 
 
@@ -249,7 +288,10 @@ def make_inputs(shape: Shape, seed: int = 0, seq_lens=None, poison: bool = True,
     else:
         num_pages = shape.batch * mpps
 
-    kv = _normal_bf16(rng, shape.pool_shape(num_pages), shape.input_scale)
+    if shape.cache_dtype == "fp8":
+        kv = _normal_e4m3(rng, shape.pool_shape(num_pages), shape.input_scale)
+    else:
+        kv = _normal_bf16(rng, shape.pool_shape(num_pages), shape.input_scale)
 
     if shape.paged:
         perm = rng.permutation(num_pages).astype(np.int32)
@@ -268,8 +310,10 @@ def make_inputs(shape: Shape, seed: int = 0, seq_lens=None, poison: bool = True,
         block_table = None
 
     if poison:
+        table = POISON_FP8 if shape.cache_dtype == "fp8" else POISON_BITS
+
         def pois(count):
-            return POISON_BITS[rng.integers(0, len(POISON_BITS), size=count)]
+            return table[rng.integers(0, len(table), size=count)]
         for p in spares:
             kv[p] = pois(kv[p].size).reshape(kv[p].shape)
         for b in range(shape.batch):
