@@ -91,6 +91,18 @@ enum kvattn_variant {
 
 enum kvattn_out_dtype { KVATTN_OUT_BF16 = 0, KVATTN_OUT_FP32 = 1 };
 
+/* Element type of the KV cache.  An fp8 cache follows the GTA/GLA page
+ * ("Mamba核心作者新作…", the 236B serving test run in FP8) and the MFA page
+ * ("突破大模型推理瓶颈…", closing paragraph: quantisation as the next step);
+ * neither fixes a format, so the reading here is e4m3 with one scale per
+ * tensor.  FP8_E4M3 (GQA with 4 heads per KV head of 128): one byte per
+ * element (sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals at
+ * exponent 0; 0x7F / 0xFF are NaN), the key is k_scale * K8, the value
+ * v_scale * V8.  The pool layout is the GQA one with byte elements
+ * ([num_pages][2][64][num_kv][128] bytes, 16-byte aligned base).  The query
+ * stays bf16 and is used as f16 inside the kernel: |q| must stay below 65504. */
+enum kvattn_cache_dtype { KVATTN_CACHE_BF16 = 0, KVATTN_CACHE_FP8_E4M3 = 1 };
+
 enum kvattn_status {
     KVATTN_OK = 0,
     KVATTN_ERR_INVALID_ARG = -1,       /* null pointer, bad size, inconsistent shape */
@@ -117,9 +129,11 @@ enum kvattn_kernel {
     KVATTN_KERNEL_LATENT_TC = 2, /* tcgen05/TMEM latent kernel, one CTA per group or branch
                                     (GLA, MLRA) */
     KVATTN_KERNEL_MQA_TC = 3,    /* tensor-core MQA kernel (one wide KV head) */
-    KVATTN_KERNEL_LATENT_PAIR = 4 /* tcgen05/TMEM MLA kernel (512 + 64) on a 2-CTA cluster:
-                                     each CTA scores half of every page and keeps half of
-                                     the value columns */
+    KVATTN_KERNEL_LATENT_PAIR = 4, /* tcgen05/TMEM MLA kernel (512 + 64) on a 2-CTA cluster:
+                                      each CTA scores half of every page and keeps half of
+                                      the value columns */
+    KVATTN_KERNEL_GQA_FP8 = 5      /* GQA over an fp8 (e4m3) cache: TMA-staged byte tiles widened
+                                      to f16 per warp, warp-level f16 MMAs, in-kernel merge */
 };
 
 /*
@@ -149,6 +163,11 @@ typedef struct {
                                   outputs side by side, [B][Q][H][R][d_nope], instead of their
                                   sum, for an up-projection with one W_UV block per branch
                                   (kvattn_head_proj) */
+    int32_t cache_dtype;       /* kvattn_cache_dtype; FP8_E4M3 only for GQA with 4 query heads
+                                  per KV head of 128 (else UNSUPPORTED) */
+    float k_scale;             /* fp8 cache: key = k_scale * stored byte value (> 0, finite) */
+    float v_scale;             /* fp8 cache: value = v_scale * stored byte value (> 0, finite);
+                                  both ignored for a bf16 cache */
 } kvattn_params;
 
 /* What kvattn_decode will launch for a problem (see kvattn_get_plan). */
@@ -348,9 +367,9 @@ int kvattn_get_device_error(const void *workspace, void *stream, int32_t *code);
 /* Static, human-readable name of a status code. */
 const char *kvattn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 201 (kvattn_params carries q_len and
- * branch_out; the steps either side: kvattn_rope, kvattn_append_kv,
- * kvattn_head_proj). */
+/* Library ABI version (major * 100 + minor): 202 (kvattn_params carries q_len,
+ * branch_out and the cache element type with its scales; the steps either side:
+ * kvattn_rope, kvattn_append_kv, kvattn_head_proj). */
 int kvattn_version(void);
 
 #ifdef __cplusplus

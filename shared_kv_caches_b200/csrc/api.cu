@@ -8,6 +8,10 @@
 #include "kvattn_internal.cuh"
 
 namespace kvattn {
+
+// The GQA kernel over an fp8 (e4m3) cache (decode_gqa_fp8.cu).
+bool gqa_fp8_supported(const Problem &pr);
+cudaError_t launch_gqa_fp8(const DecodeArgs &a, float k_scale, float v_scale, cudaStream_t st);
 namespace {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -31,6 +35,14 @@ int validate(int32_t variant, const kvattn_params *p, Problem *pr)
         return KVATTN_ERR_INVALID_ARG;
     if (p->branch_out != 0 && (p->branch_out != 1 || variant != KVATTN_MLRA))
         return KVATTN_ERR_INVALID_ARG;
+    if (p->cache_dtype != KVATTN_CACHE_BF16 && p->cache_dtype != KVATTN_CACHE_FP8_E4M3)
+        return KVATTN_ERR_INVALID_ARG;
+    if (p->cache_dtype == KVATTN_CACHE_FP8_E4M3) {
+        if (!(p->k_scale > 0.f) || !(p->v_scale > 0.f) || !isfinite(p->k_scale) || !isfinite(p->v_scale))
+            return KVATTN_ERR_INVALID_ARG;
+        if (variant != KVATTN_GQA)
+            return KVATTN_ERR_UNSUPPORTED;
+    }
     const int q_len = p->q_len > 0 ? p->q_len : 1;
     if (q_len > kMaxQueryLen || (long long)p->batch * q_len > 65535 || p->num_q_heads > 65535)
         return KVATTN_ERR_UNSUPPORTED;
@@ -201,6 +213,24 @@ int make_plan(const Problem &pr, int forced_splits, Plan *pl)
     return KVATTN_OK;
 }
 
+// The plan of a call: the cache element type picks the kernel for the same
+// geometry (an fp8 cache has its own GQA kernel; other shapes are refused).
+int plan_call(const kvattn_params *p, const Problem &pr, Plan *pl)
+{
+    if (p->cache_dtype == KVATTN_CACHE_FP8_E4M3 && !gqa_fp8_supported(pr))
+        return KVATTN_ERR_UNSUPPORTED;
+    const int st = make_plan(pr, p->num_splits, pl);
+    if (st)
+        return st;
+    if (p->cache_dtype == KVATTN_CACHE_FP8_E4M3) {
+        // same grid, parts and in-kernel merge as the bf16 GQA plan
+        if (pl->pub.kernel != KVATTN_KERNEL_GQA || !pl->fused_merge)
+            return KVATTN_ERR_UNSUPPORTED;
+        pl->pub.kernel = KVATTN_KERNEL_GQA_FP8;
+    }
+    return KVATTN_OK;
+}
+
 }  // namespace
 
 int sm_count()
@@ -249,7 +279,7 @@ int validate_call(int32_t variant, const kvattn_params *p, const void *q_nope, c
 
 using namespace kvattn;
 
-extern "C" int kvattn_version(void) { return 201; }
+extern "C" int kvattn_version(void) { return 202; }
 
 extern "C" const char *kvattn_status_string(int status)
 {
@@ -273,7 +303,7 @@ extern "C" int kvattn_get_plan(int32_t variant, const kvattn_params *p, kvattn_p
     if (st)
         return st;
     Plan pl;
-    st = make_plan(pr, p->num_splits, &pl);
+    st = plan_call(p, pr, &pl);
     if (st)
         return st;
     *plan = pl.pub;
@@ -315,7 +345,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     if (st)
         return st;
     Plan pl;
-    st = make_plan(pr, p->num_splits, &pl);
+    st = plan_call(p, pr, &pl);
     if (st)
         return st;
     if (workspace_bytes < pl.pub.workspace_bytes)
@@ -365,6 +395,7 @@ extern "C" int kvattn_decode_timed(int32_t variant, const kvattn_params *p, cons
     cudaError_t le;
     switch (pl.pub.kernel) {
     case KVATTN_KERNEL_GQA: le = launch_gqa(a, s); break;
+    case KVATTN_KERNEL_GQA_FP8: le = launch_gqa_fp8(a, p->k_scale, p->v_scale, s); break;
     case KVATTN_KERNEL_MQA_TC: le = launch_mqa_mma(a, s); break;
     case KVATTN_KERNEL_LATENT_TC: le = launch_latent_tc(a, pr, s); break;
     case KVATTN_KERNEL_LATENT_PAIR: le = launch_latent_pair(a, s); break;

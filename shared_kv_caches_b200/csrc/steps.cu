@@ -344,6 +344,8 @@ extern "C" int kvattn_append_kv(int32_t variant, const kvattn_params *p, const v
         return st;
     if (!new_kv || !pos || !kv_cache)
         return KVATTN_ERR_INVALID_ARG;
+    if (p->cache_dtype != KVATTN_CACHE_BF16)
+        return KVATTN_ERR_UNSUPPORTED;      // rows are appended in bf16
     if (!(rope_base == 0.f || (rope_base > 1.f && isfinite(rope_base))))
         return KVATTN_ERR_INVALID_ARG;
     if (!is_aligned(new_kv, 16) || !is_aligned(kv_cache, 16) || !is_aligned(pos, 4) ||

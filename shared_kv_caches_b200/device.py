@@ -26,7 +26,10 @@ class DeviceProblem:
         self.variant = K.VARIANTS[s.variant]
         self.q_nope = bf16_tensor(inputs["q_nope"], self.device)
         self.q_rope = None if inputs["q_rope"] is None else bf16_tensor(inputs["q_rope"], self.device)
-        self.kv = bf16_tensor(inputs["kv"], self.device)
+        if getattr(s, "cache_dtype", "bf16") == "fp8":
+            self.kv = torch.from_numpy(np.ascontiguousarray(inputs["kv"], dtype=np.uint8)).to(self.device)
+        else:
+            self.kv = bf16_tensor(inputs["kv"], self.device)
         bt = inputs["block_table"]
         self.block_table = None if bt is None else torch.from_numpy(bt).to(self.device)
         self.seq_lens = torch.from_numpy(np.asarray(inputs["seq_lens"], np.int32)).to(self.device)

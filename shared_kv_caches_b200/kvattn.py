@@ -32,7 +32,8 @@ KVATTN_DEVERR_PAGE_OUT_OF_RANGE = 1
 KVATTN_DEVERR_SEQ_TOO_LONG = 2
 KVATTN_DEVERR_WAIT_TIMEOUT = 4
 KVATTN_DEVERR_POS_OUT_OF_RANGE = 8
-KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc", 4: "latent_pair"}
+KERNEL_NAMES = {0: "generic", 1: "gqa", 2: "latent_tc", 3: "mqa_tc", 4: "latent_pair", 5: "gqa_fp8"}
+KVATTN_CACHE_BF16, KVATTN_CACHE_FP8_E4M3 = 0, 1
 KVATTN_SELFTEST_MISSED_PHASE = 256
 
 EXPORTS = ("kvattn_get_plan", "kvattn_workspace_size", "kvattn_workspace_init", "kvattn_decode",
@@ -45,7 +46,8 @@ KVATTN_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 class kvattn_params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "num_q_heads", "num_kv", "d_nope", "d_rope", "page_size", "max_pages_per_seq",
-        "num_pages", "max_seq_len", "num_splits", "out_dtype", "q_len", "branch_out")]
+        "num_pages", "max_seq_len", "num_splits", "out_dtype", "q_len", "branch_out", "cache_dtype")] + [
+        ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 class kvattn_plan(ctypes.Structure):
@@ -101,10 +103,11 @@ def load():
 
 def make_params(batch, num_q_heads, num_kv, d_nope, d_rope, max_pages_per_seq, num_pages,
                 max_seq_len, num_splits=0, out_dtype=KVATTN_OUT_BF16, page_size=64, q_len=1,
-                branch_out=0) -> kvattn_params:
+                branch_out=0, cache_dtype=0, k_scale=1.0, v_scale=1.0) -> kvattn_params:
     return kvattn_params(int(batch), int(num_q_heads), int(num_kv), int(d_nope), int(d_rope),
                          int(page_size), int(max_pages_per_seq), int(num_pages), int(max_seq_len),
-                         int(num_splits), int(out_dtype), int(q_len), int(branch_out))
+                         int(num_splits), int(out_dtype), int(q_len), int(branch_out), int(cache_dtype),
+                         float(k_scale), float(v_scale))
 
 
 def kvattn_version() -> int:
@@ -185,7 +188,9 @@ def params_for(shape, max_pages_per_seq, num_pages, max_seq_len, num_splits=0) -
     return make_params(shape.batch, shape.num_q_heads, shape.num_kv, shape.d_nope, shape.d_rope,
                        max_pages_per_seq, num_pages, max_seq_len, num_splits,
                        KVATTN_OUT_FP32 if shape.out_dtype == "fp32" else KVATTN_OUT_BF16,
-                       shape.page_size, shape.q_len, 1 if getattr(shape, "branch_out", False) else 0)
+                       shape.page_size, shape.q_len, 1 if getattr(shape, "branch_out", False) else 0,
+                       KVATTN_CACHE_FP8_E4M3 if getattr(shape, "cache_dtype", "bf16") == "fp8" else KVATTN_CACHE_BF16,
+                       getattr(shape, "k_scale", 1.0), getattr(shape, "v_scale", 1.0))
 
 
 def decode_tensors(variant, params, q_nope, q_rope, kv, block_table, seq_lens, sm_scale, out, lse,

@@ -54,7 +54,9 @@ def _params(name, **kw):
     mpps = (hi + 63) // 64
     p = dict(batch=s.batch, num_q_heads=s.num_q_heads, num_kv=s.num_kv, d_nope=s.d_nope, d_rope=s.d_rope,
              max_pages_per_seq=mpps, num_pages=mpps * s.batch + 1, max_seq_len=hi, num_splits=0,
-             out_dtype=1 if s.out_dtype == "fp32" else 0)
+             out_dtype=1 if s.out_dtype == "fp32" else 0,
+             cache_dtype=K.KVATTN_CACHE_FP8_E4M3 if s.cache_dtype == "fp8" else K.KVATTN_CACHE_BF16,
+             k_scale=s.k_scale, v_scale=s.v_scale)
     p.update(kw)
     return s, K.make_params(**p)
 
@@ -79,6 +81,7 @@ def test_plan_every_workload(lib, name):
 EXPECTED_PLANS = {
     "gla": ("latent_tc", 4, 64, 512, 2),
     "gqa": ("gqa", 7, 19, 1792, 1),
+    "gqa_fp8": ("gqa_fp8", 7, 19, 1792, 1),
     "mfa": ("mqa_tc", 6, 22, 192, 2),
     "mla": ("latent_pair", 5, 103, 640, 2),
     "mlra_128k": ("latent_tc", 37, 56, 148, 2),
@@ -164,6 +167,28 @@ def test_small_workspace_rejected(lib):
     s, p = _params("mla")
     need = K.kvattn_workspace_size(s.variant_id, p)
     assert _decode(s.variant_id, p, ws_bytes=need - 1) == K.KVATTN_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("k_scale", 0.0, K.KVATTN_ERR_INVALID_ARG),
+    ("k_scale", -1.0, K.KVATTN_ERR_INVALID_ARG),
+    ("v_scale", float("nan"), K.KVATTN_ERR_INVALID_ARG),
+    ("v_scale", float("inf"), K.KVATTN_ERR_INVALID_ARG),
+    ("cache_dtype", 2, K.KVATTN_ERR_INVALID_ARG),
+    ("d_nope", 64, K.KVATTN_ERR_UNSUPPORTED),           # the fp8 kernel holds 128-dim heads
+    ("num_kv", 16, K.KVATTN_ERR_UNSUPPORTED),           # 2 query heads per KV head
+])
+def test_bad_fp8_params_rejected(lib, field, value, status):
+    s, p = _params("gqa_fp8", **{field: value})
+    assert _decode(s.variant_id, p) == status
+
+
+@pytest.mark.parametrize("name", ["mfa", "mla", "gla", "mlra_128k", "gta"])
+def test_fp8_cache_only_for_gqa(lib, name):
+    s, p = _params(name, cache_dtype=K.KVATTN_CACHE_FP8_E4M3, k_scale=1.0, v_scale=1.0)
+    assert _decode(s.variant_id, p) == K.KVATTN_ERR_UNSUPPORTED
+    with pytest.raises(K.KvattnError):
+        K.kvattn_get_plan(s.variant_id, p)
 
 
 def test_non_finite_scale_rejected(lib):

@@ -87,6 +87,10 @@ SMALL = {
     "gta": (W.WORKLOADS["gta"].replace(batch=3, ctx=(1, 700)), None),
     "mfa_kr": (W.WORKLOADS["mfa_kr"].replace(batch=3, ctx=(1, 700)), None),
     "gta_generic": (W.WORKLOADS["gta"].replace(batch=2, num_q_heads=8, num_kv=2, d_nope=64, ctx=(1, 300)), None),
+    # fp8 (e4m3) cache with per-tensor scales, and with unit scales
+    "gqa_fp8": (W.WORKLOADS["gqa_fp8"].replace(batch=3, ctx=(1, 700)), None),
+    "gqa_fp8_unit_scales": (W.WORKLOADS["gqa_fp8"].replace(batch=3, ctx=(1, 700), k_scale=1.0, v_scale=1.0), None),
+    "gqa_fp8_contiguous": (W.WORKLOADS["gqa_fp8"].replace(batch=2, ctx=(1, 300), paged=False), None),
 }
 
 
@@ -109,6 +113,7 @@ SWEEP_SHAPES = {
     "mlra": W.WORKLOADS["mlra_128k"],
     "gta": W.WORKLOADS["gta"],
     "mfa_kr": W.WORKLOADS["mfa_kr"],
+    "gqa_fp8": W.WORKLOADS["gqa_fp8"],
 }
 
 
@@ -142,7 +147,7 @@ def _sample(x, shape):
 
 
 @pytest.mark.parametrize("name", ["gqa", "mfa", "mla", "gla", "mlra_128k", "mlra_512k", "mlra_1m",
-                                  "mlra_b8_128k", "gta", "mfa_kr"])
+                                  "mlra_b8_128k", "gta", "mfa_kr", "gqa_fp8"])
 def test_parity_full_size_sampled(dev, oracle_mod, name):
     """Full benchmark sizes, library-chosen launch (as timed by bench.py);
     the oracle computes sampled sequences (and heads for batch 1)."""
@@ -166,6 +171,7 @@ def test_benchmark_shapes_use_the_specialised_kernels(dev):
     assert kernel_of(W.WORKLOADS["tiny_mla"]) == "generic"
     assert kernel_of(W.WORKLOADS["gta"]) == "gqa"
     assert kernel_of(W.WORKLOADS["mfa_kr"]) == "mqa_tc"
+    assert kernel_of(W.WORKLOADS["gqa_fp8"]) == "gqa_fp8"
     assert kernel_of(SMALL["gta_generic"][0]) == "generic"
     for name in ("gla1_shard", "gla4", "gla8", "mlra1_shard", "mlra2", "mlra8"):
         assert kernel_of(SMALL[name][0]) == "latent_tc", name
@@ -193,7 +199,7 @@ def _repermute(x, seed):
     return dict(x, kv=kv2, block_table=newpos[x["block_table"]])
 
 
-@pytest.mark.parametrize("name", ["gqa", "mla", "mlra"])
+@pytest.mark.parametrize("name", ["gqa", "mla", "mlra", "gqa_fp8"])
 def test_block_table_permutation_is_bit_identical(dev, name):
     shape = SWEEP_SHAPES[name].replace(batch=3, ctx=(500, 3000))
     x = W.make_inputs(shape, seed=3)
@@ -214,6 +220,37 @@ def test_poison_outside_context_changes_nothing(dev, name):
     _, out2, lse2 = run_gpu(dict(x, kv=kv), dev)
     np.testing.assert_array_equal(out1, out2)
     np.testing.assert_array_equal(lse1, lse2)
+
+
+def test_poison_outside_context_changes_nothing_fp8(dev):
+    """fp8 cache: NaN and +-448 codes past each context swapped for one another."""
+    shape = SWEEP_SHAPES["gqa_fp8"].replace(batch=3, ctx=(65, 1000))
+    x = W.make_inputs(shape, seed=4)
+    _, out1, lse1 = run_gpu(x, dev)
+    kv = x["kv"].copy()
+    pois = np.isin(kv, W.POISON_FP8)
+    kv[pois] = np.where(kv[pois] == 0x7F, 0x7E, 0x7F).astype(np.uint8)
+    _, out2, lse2 = run_gpu(dict(x, kv=kv), dev)
+    np.testing.assert_array_equal(out1, out2)
+    np.testing.assert_array_equal(lse1, lse2)
+
+
+def test_context_of_one_returns_scaled_value_fp8(dev, oracle_mod):
+    """ctx = 1 over an fp8 cache: the output is v_scale times the decoded value
+    row, exactly (an e4m3 value times a power of two fits bf16)."""
+    import torch
+    shape = SWEEP_SHAPES["gqa_fp8"].replace(batch=2, ctx=(1, 1))
+    x = W.make_inputs(shape, seed=7)
+    p, _, _ = run_gpu(x, dev)
+    got = p.out.view(dtype=torch.int16).cpu().numpy().view(np.uint16)
+    g_of = np.arange(shape.num_q_heads) // (shape.num_q_heads // shape.num_kv)
+    for b in range(2):
+        page, slot = W.token_location(x, b, 0)
+        # + 0.0: a -0 code comes out as +0 (the accumulators start at +0)
+        want = shape.v_scale * oracle_mod.e4m3_value(x["kv"][page, 1, slot, g_of]) + 0.0
+        bits = (want.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        assert np.array_equal(want.astype(np.float32).view(np.uint32) & 0xFFFF, np.zeros_like(bits))
+        np.testing.assert_array_equal(got[b], bits)
 
 
 def test_split_count_changes_only_rounding(dev):
@@ -344,6 +381,7 @@ Q_SHAPES = {
     "mlra": W.WORKLOADS["mlra_128k"].replace(batch=2, ctx=(100, 700)),
     "tiny_mla": W.WORKLOADS["tiny_mla"],
     "gta": W.WORKLOADS["gta"].replace(batch=3, ctx=(1, 700)),
+    "gqa_fp8": W.WORKLOADS["gqa_fp8"].replace(batch=3, ctx=(1, 700)),
 }
 
 
