@@ -10,16 +10,25 @@
 // softmax scale; outputs are v_scale * sum_j p_j V8_j: the scale multiplies
 // the normalised part output.
 //
-// Layout and roles follow the bf16 GQA kernel: a producer warp streams each
-// page's K and V tiles (64 tokens x 128 bytes each, one TMA box with the
-// 128-byte swizzle) into a two-stage ring; four consumer warps each own 16
-// tokens of a page.  A warp first widens its 16 rows of K and V to f16
-// (cvt.rn.f16x2.e4m3x2: e4m3 values are exactly representable in f16) into
-// a CTA-wide 16-bit tile with the bf16 kernel's swizzled layout, zeroing rows
-// past the context, and releases the fp8 stage at once; then the transposed
-// warp-level MMAs run as in the bf16 kernel, in f16 (m16n8k16, fp32
-// accumulate) with the query converted to f16 once.  The last CTA of each
-// (sequence, KV head) merges the parts.
+// A producer warp streams each page's K and V tiles (64 tokens x 128 bytes
+// each, one TMA box with the 128-byte swizzle) into a four-stage ring (the
+// byte tiles are half the size of bf16 ones, so twice the stages keep as
+// many bytes in flight); four consumer warps each own 16 tokens of a page.
+// Each lane loads its bytes of the warp's K and V rows straight into
+// registers (16-byte loads, conflict-free under the swizzle), the warp
+// releases the stage at once, and the bytes become the f16 fragments of the
+// transposed warp-level MMAs in registers (cvt.rn.f16x2.e4m3x2: e4m3 values
+// are exactly representable in f16):
+//  - S^T = K Q^T contracts over the head dims, so the dims may take any
+//    order that K and Q share: step kk = 4s + w of lane (r, c) holds dims
+//    32c + 16s + 4w .. +3, which is the 16-byte chunk 2c + s of rows r and
+//    r + 8, read whole;
+//  - O^T = V^T P^T contracts over tokens and its rows are output dims: lane
+//    (r, c) reads chunk r (dims 16r .. 16r + 15) of its four tokens 2c, 2c+1,
+//    8+2c, 9+2c and pairs the tokens byte by byte (prmt); row r of M-tile mt
+//    is then dim 16r + 4(mt/2) + 2(mt%2), row r + 8 the next dim.
+// The query (bf16) is used as f16, loaded once in the dims' order.  The last
+// CTA of each (sequence, KV head) merges the parts.
 #include <math.h>
 
 #include <cuda_fp16.h>
@@ -34,18 +43,15 @@ namespace {
 constexpr int D = 128;
 constexpr int G = 4;
 constexpr int CW = 4;                        // consumer warps
-constexpr int STAGES = 2;
+constexpr int STAGES = 4;
 constexpr int TPW = kPage / CW;              // tokens per warp per page
 constexpr int THREADS = (CW + 1) * 32;
 constexpr int TILE8 = kPage * D;             // fp8 K (or V) tile: 64 tokens x 128 bytes, one swizzle span
 constexpr int STAGE8 = 2 * TILE8;            // K and V
-constexpr int BOX_BYTES = kPage * 64 * 2;    // 16-bit tile: 64 tokens x 64 dims per 128-byte swizzle span
-constexpr int TILE_BYTES = 2 * BOX_BYTES;    // 64 tokens x 128 dims
 constexpr float kLn2 = 0.69314718055994531f;
 
 struct Fp8Smem {
     unsigned char tiles[STAGES][STAGE8];        // fp8 stages (1024-byte aligned, swizzle atoms)
-    unsigned char wide[2][TILE_BYTES];          // K and V widened to f16, each warp its own 16 rows
     float ow[CW][G][D];                         // per-warp outputs for the final merge
     float mw[CW][G];
     float lw[CW][G];
@@ -55,16 +61,10 @@ struct Fp8Smem {
     int last;
 };
 
-// Byte offset of 16-byte chunk c (8 dims) of token row t in a swizzled 16-bit tile.
-__device__ __forceinline__ uint32_t chunk_off(int t, int c)
+// Word i (compile-time after unrolling) of a 16-byte load.
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 {
-    return (uint32_t)((c >> 3) * BOX_BYTES + t * 128 + (((c & 7) ^ (t & 7)) << 4));
-}
-
-// Byte offset of 16-byte chunk c (16 dims) of token row t in a swizzled fp8 tile.
-__device__ __forceinline__ uint32_t chunk8_off(int t, int c)
-{
-    return (uint32_t)(t * 128 + ((c ^ (t & 7)) << 4));
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 // Two e4m3 bytes (low byte first) to two f16 (low half first), exactly.
@@ -74,20 +74,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v)
     const uint16_t h = (uint16_t)(v & 0xffffu);
     asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "h"(h));
     return r;
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
 }
 
 // c (16 x 8, fp32) += a (16 x 16, f16, row) * b (16 x 8, f16, col)
@@ -175,19 +161,21 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_fp8_decode_kernel(const __grid
     }
 
     // ---------------------------------------------------------------- consumers
-    // fragment coordinates: r = row group (token of S^T, dim of O^T, head of
+    // fragment coordinates: r = row group (token of S^T, dims of O^T, head of
     // the B operands), c = column pair (heads 2c, 2c+1 of S^T and O^T; only
     // c < 2 are real heads)
     const int r = lane >> 2, c = lane & 3;
-    const int mrow = lane & 7, mat = lane >> 3;
-    // Q^T as the B operand of S^T = K Q^T: b0 = dims 16kk + 2c.., b1 = + 8, head r
+    // Q^T as the B operand of S^T = K Q^T (head r) in the dims' order of the
+    // K fragments: step kk = 4s + w holds dims 32c + 16s + 4w + {0, 1} (b0)
+    // and + {2, 3} (b1)
     uint32_t qb[D / 16][2];
     {
-        const __nv_bfloat16 *qr = a.q_nope + ((size_t)b * a.H + kvh * G + (r < G ? r : 0)) * D;
+        const __nv_bfloat16 *qr = a.q_nope + ((size_t)b * a.H + kvh * G + (r < G ? r : 0)) * D + 32 * c;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-            qb[kk][0] = r < G ? bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qr + 16 * kk + 2 * c)) : 0u;
-            qb[kk][1] = r < G ? bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qr + 16 * kk + 8 + 2 * c)) : 0u;
+            const int d = 16 * (kk >> 2) + 4 * (kk & 3);
+            qb[kk][0] = r < G ? bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qr + d)) : 0u;
+            qb[kk][1] = r < G ? bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qr + d + 2)) : 0u;
         }
     }
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2c, 2c+1
@@ -206,41 +194,40 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_fp8_decode_kernel(const __grid
         }
         const int ntok = min(kPage, L - (p0 + i) * kPage);
         const int nw = S.skip[st] ? 0 : min(max(ntok - t0, 0), TPW);
+        // this lane's bytes of the warp's rows: row t of a tile sits at t * 128
+        // with its 16-byte chunk j at (j ^ (t & 7)) * 16; t0 is a multiple of 8
+        uint4 kr[2][2], vr[4];
         if (nw > 0) {
-            // widen this warp's 16 rows of K and V to f16 (rows past the
-            // context become zeros: 0 * NaN would poison the MMA)
-#pragma unroll 2
-            for (int idx = lane; idx < 2 * TPW * (D / 16); idx += 32) {
-                const int plane = idx / (TPW * (D / 16)), rem = idx % (TPW * (D / 16));
-                const int row = rem / (D / 16), c16 = rem % (D / 16);
-                const int t = t0 + row;
-                uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-                if (row < nw) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(S.tiles[st] + plane * TILE8 + chunk8_off(t, c16));
-                    lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16), e4m3x2_to_f16x2(v.y),
-                                    e4m3x2_to_f16x2(v.y >> 16));
-                    hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16), e4m3x2_to_f16x2(v.w),
-                                    e4m3x2_to_f16x2(v.w >> 16));
-                }
-                *reinterpret_cast<uint4 *>(S.wide[plane] + chunk_off(t, 2 * c16)) = lo;
-                *reinterpret_cast<uint4 *>(S.wide[plane] + chunk_off(t, 2 * c16 + 1)) = hi;
+            const unsigned char *kt = S.tiles[st] + t0 * 128, *vt = kt + TILE8;
+            // K: chunk 2c + s of rows r and r + 8
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int off = ((2 * c + s2) ^ r) << 4;
+                kr[s2][0] = *reinterpret_cast<const uint4 *>(kt + r * 128 + off);
+                kr[s2][1] = *reinterpret_cast<const uint4 *>(kt + (r + 8) * 128 + off);
+            }
+            // V: chunk r of tokens 2c, 2c + 1, 8 + 2c, 9 + 2c; tokens past the
+            // context become zeros (0 * NaN would poison the MMA)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = 2 * c + (j & 1) + ((j >> 1) << 3);
+                vr[j] = t < nw ? *reinterpret_cast<const uint4 *>(vt + t * 128 + ((r ^ (t & 7)) << 4))
+                               : make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        // the fp8 stage is free for the next TMA load once every lane read its rows
+        // the stage is free for the next TMA load once every lane holds its bytes
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&S.empty[st]);
         if (nw > 0) {
-            unsigned char *Kb = S.wide[0];
-            unsigned char *Vb = S.wide[1];
-            const uint32_t kbase = smem_u32(Kb), vbase = smem_u32(Vb);
-            // S^T (16 tokens x 8 head columns) = K Q^T
+            // S^T (16 tokens x 8 head columns) = K Q^T; a0/a2 = row r, a1/a3 =
+            // row r + 8, low/high byte pair of one word = dims + {0, 1} / + {2, 3}
             float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(kbase + chunk_off(t0 + ((mat & 1) << 3) + mrow, 2 * kk + (mat >> 1)), a0, a1, a2, a3);
-                mma_f16(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+                const uint32_t w0 = word_of(kr[kk >> 2][0], kk & 3), w1 = word_of(kr[kk >> 2][1], kk & 3);
+                mma_f16(s, e4m3x2_to_f16x2(w0), e4m3x2_to_f16x2(w1), e4m3x2_to_f16x2(w0 >> 16),
+                        e4m3x2_to_f16x2(w1 >> 16), qb[kk][0], qb[kk][1]);
             }
             // online softmax per head over the warp's tokens (rows r and r + 8)
             float mx[2];
@@ -280,17 +267,24 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_fp8_decode_kernel(const __grid
             const uint32_t pb0 = movm_t(pack_f16(p[0], p[1]));
             const uint32_t pb1 = movm_t(pack_f16(p[2], p[3]));
 #pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                o[mt][0] *= alpha[0];
-                o[mt][1] *= alpha[1];
-                o[mt][2] *= alpha[0];
-                o[mt][3] *= alpha[1];
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(vbase + chunk_off(t0 + ((mat >> 1) << 3) + mrow, 2 * mt + (mat & 1)), a0, a1, a2, a3);
-                mma_f16(o[mt], a0, a1, a2, a3, pb0, pb1);
+            for (int w = 0; w < 4; ++w) {
+                // byte pairs of tokens (2c, 2c + 1) and (8 + 2c, 9 + 2c), dims 16r + 4w .. + 3
+                const uint32_t x0 = word_of(vr[0], w), x1 = word_of(vr[1], w);
+                const uint32_t x2 = word_of(vr[2], w), x3 = word_of(vr[3], w);
+                const uint32_t lo01 = __byte_perm(x0, x1, 0x5140), hi01 = __byte_perm(x0, x1, 0x7362);
+                const uint32_t lo23 = __byte_perm(x2, x3, 0x5140), hi23 = __byte_perm(x2, x3, 0x7362);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    o[2 * w][e] *= alpha[e & 1];
+                    o[2 * w + 1][e] *= alpha[e & 1];
+                }
+                // M-tile 2w: rows r / r + 8 = dims 16r + 4w / + 1; M-tile 2w + 1: + 2 / + 3
+                mma_f16(o[2 * w], e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(lo23),
+                        e4m3x2_to_f16x2(lo23 >> 16), pb0, pb1);
+                mma_f16(o[2 * w + 1], e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi01 >> 16), e4m3x2_to_f16x2(hi23),
+                        e4m3x2_to_f16x2(hi23 >> 16), pb0, pb1);
             }
         }
-        __syncwarp();   // this warp's f16 rows are rewritten on the next page
     }
 
     // merge the four warps' states and write this part's result
@@ -303,10 +297,12 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_fp8_decode_kernel(const __grid
             }
         }
 #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt)
+        for (int mt = 0; mt < D / 16; ++mt) {
+            const int d0 = 16 * r + 4 * (mt >> 1) + 2 * (mt & 1);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                S.ow[warp][2 * c + (e & 1)][16 * mt + r + ((e >> 1) << 3)] = o[mt][e];
+                S.ow[warp][2 * c + (e & 1)][d0 + (e >> 1)] = o[mt][e];
+        }
     }
     named_sync(1, CW * 32);
 
