@@ -468,7 +468,7 @@ def run_ours(args, rank, world, local):
                                                      "gpu_launches")}
             for r in results}
     if args.workload == "suite" and world == 1 and not args.no_steps:
-        line["steps"] = measure_steps(args, dev, peaks, flush)
+        line["steps_ops"] = measure_steps(args, dev, peaks, flush)
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if world > 1:

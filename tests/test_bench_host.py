@@ -39,6 +39,14 @@ def test_stored_traffic_matches_only_current_digest():
     assert bench.stored_traffic("no-such-workload", "x", rows[0][4]) is None
 
 
+def test_line_keeps_the_timed_step_count():
+    """"steps" in the JSON line is the timed step count K; the breakdown of
+    the steps either side of attention goes under its own key."""
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert 'line["steps"] =' not in src
+    assert 'line["steps_ops"] = measure_steps' in src
+
+
 def test_suite_covers_every_benchmark_problem():
     """The default run times every benchmark problem except the tiny parity
     case, with MLA (the largest single-GPU problem) as the headline."""
