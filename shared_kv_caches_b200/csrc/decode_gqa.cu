@@ -46,9 +46,9 @@ struct GqaSmem {
     float ow[CW][G][D];                         // per-warp outputs for the final merge
     float mw[CW][G];
     float lw[CW][G];
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    int skip[STAGES];
+    uint64_t full[2 * STAGES];                  // one per slot (tied pages: two slots per stage)
+    uint64_t empty[2 * STAGES];
+    int skip[2 * STAGES];
     int last;
 };
 
@@ -97,6 +97,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// TIED: one plane per page that serves as key and value (GTA)
+template <bool TIED>
 __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_constant__ CUtensorMap kv_map,
                                                              const DecodeArgs a)
 {
@@ -110,8 +112,15 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
     const int p0 = split * a.pages_per_split;
     const int n = max(0, min(npages, p0 + a.pages_per_split) - p0);
 
+    // tied keys and values (GTA) fill half a stage per page: the ring then
+    // holds twice as many one-tile slots, so as many bytes stay in flight
+    constexpr bool tied = TIED;
+    constexpr int nslots = tied ? 2 * STAGES : STAGES;
+    constexpr int slot_bytes = tied ? TILE_BYTES : STAGE_BYTES;
+    unsigned char *const ring = &S.tiles[0][0];
+
     if (threadIdx.x == 0) {
-        for (int st = 0; st < STAGES; ++st) {
+        for (int st = 0; st < nslots; ++st) {
             mbar_init(&S.full[st], 1);
             mbar_init(&S.empty[st], CW);
         }
@@ -124,8 +133,8 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
         if (lane == 0 && n > 0) {
             prefetch_tmap(&kv_map);
             for (int i = 0; i < n; ++i) {
-                const int st = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&S.empty[st], ((i / STAGES) - 1) & 1)) {
+                const int st = i % nslots;
+                if (i >= nslots && !mbar_wait(&S.empty[st], ((i / nslots) - 1) & 1)) {
                     raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
                     break;
                 }
@@ -138,11 +147,10 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
                     continue;
                 }
                 S.skip[st] = 0;
-                // tied keys and values (GTA): one tile serves as both
-                const bool tied = a.kv_planes == 1;
+                // tied: one tile serves as key and value
                 mbar_arrive_expect_tx(&S.full[st], tied ? TILE_BYTES : STAGE_BYTES);
                 const int zk = (int)(page * a.kv_planes * kPage), zv = zk + kPage;
-                unsigned char *t = S.tiles[st];
+                unsigned char *t = ring + (size_t)st * slot_bytes;
                 tma_load_3d(t, &kv_map, 0, kvh, zk, &S.full[st]);
                 tma_load_3d(t + BOX_BYTES, &kv_map, 64, kvh, zk, &S.full[st]);
                 if (!tied) {
@@ -178,8 +186,8 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
 
     const int t0 = warp * TPW;
     for (int i = 0; i < n; ++i) {
-        const int st = i % STAGES;
-        if (!mbar_wait(&S.full[st], (i / STAGES) & 1)) {
+        const int st = i % nslots;
+        if (!mbar_wait(&S.full[st], (i / nslots) & 1)) {
             if (lane == 0)
                 raise_error(a.err, KVATTN_DEVERR_WAIT_TIMEOUT);
             break;
@@ -187,8 +195,8 @@ __global__ void __launch_bounds__(THREADS, 3) gqa_decode_kernel(const __grid_con
         const int ntok = min(kPage, L - (p0 + i) * kPage);
         const int nw = S.skip[st] ? 0 : min(max(ntok - t0, 0), TPW);
         if (nw > 0) {
-            unsigned char *Kb = S.tiles[st];
-            unsigned char *Vb = a.kv_planes == 1 ? Kb : Kb + TILE_BYTES;
+            unsigned char *Kb = ring + (size_t)st * slot_bytes;
+            unsigned char *Vb = tied ? Kb : Kb + TILE_BYTES;
             if (nw < TPW) {
                 // value rows of this warp past the context: 0 * NaN would poison the MMA
                 for (int idx = lane; idx < (TPW - nw) * (D / 8); idx += 32)
@@ -328,10 +336,11 @@ cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t st)
                      box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const size_t smem = gqa_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = a.kv_planes == 1 ? gqa_decode_kernel<true> : gqa_decode_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    gqa_decode_kernel<<<dim3(a.num_splits, a.NU, a.B), THREADS, smem, st>>>(map, a);
+    kern<<<dim3(a.num_splits, a.NU, a.B), THREADS, smem, st>>>(map, a);
     return cudaGetLastError();
 }
 
