@@ -47,6 +47,18 @@ def test_line_keeps_the_timed_step_count():
     assert 'line["steps_ops"] = measure_steps' in src
 
 
+def test_cache_bytes_per_token_of_each_variant():
+    """Algorithmic cache bytes per context token: K and V of every KV head in
+    bf16 (one byte per element for the fp8 cache), one tied plane for GTA and
+    MFA-KR, the 576-wide latent row for MLA, GLA-2 and MLRA-4."""
+    from shared_kv_caches_b200 import benchutil as BU
+    from shared_kv_caches_b200 import workloads as W
+    want = {"gqa": 4096, "gqa_fp8": 2048, "gta": 2048, "mfa": 1024, "mfa_kr": 512, "mla": 1152, "gla": 1152,
+            "mlra_128k": 1152}
+    for name, n in want.items():
+        assert BU.kv_bytes_per_token(W.WORKLOADS[name]) == n, name
+
+
 def test_suite_covers_every_benchmark_problem():
     """The default run times every benchmark problem except the tiny parity
     case, with MLA (the largest single-GPU problem) as the headline."""

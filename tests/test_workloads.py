@@ -15,6 +15,47 @@ def test_bf16_round_to_nearest_even():
     assert back[3] == -2.5 and back[4] == 9984.0
 
 
+def test_e4m3_round_to_nearest_even_and_saturate():
+    e = W.f32_to_e4m3_bits
+    # 1 + 2^-4 is a tie between 1.0 (0x38) and 1.125 (0x39): the even code wins;
+    # 1 + 3 * 2^-4 ties 1.125 and 1.25: 0x3A
+    assert list(e([1.0625, 1.0625 + 1e-6, 1.1875, -1.0625])) == [0x38, 0x39, 0x3A, 0xB8]
+    # subnormals are multiples of 2^-9: 2^-10 ties 0 and 2^-9, 3 * 2^-10 and
+    # 5 * 2^-10 tie onto 2 * 2^-9; 7.75 * 2^-9 rounds up to the smallest normal
+    assert list(e([2.0 ** -10, 3 * 2.0 ** -10, 5 * 2.0 ** -10, 7.75 * 2.0 ** -9])) == [0x00, 0x02, 0x02, 0x08]
+    assert list(e([448.0, 460.0, 1e9, np.inf, -np.inf])) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    assert e(np.nan) == 0x7F
+    assert e(0.0) == 0x00 and e(-0.0) == 0x80
+
+
+def test_e4m3_midpoints_between_every_pair_of_codes(oracle_mod):
+    """Brute force over the format: halfway between neighbouring finite codes
+    goes to the even code, a little above halfway to the upper one."""
+    codes = np.arange(0x7E)
+    lo, hi = oracle_mod.e4m3_value(codes), oracle_mod.e4m3_value(codes + 1)
+    mid = (lo + hi) / 2
+    even = np.where(codes % 2 == 0, codes, codes + 1)
+    np.testing.assert_array_equal(W.f32_to_e4m3_bits(mid), even)
+    np.testing.assert_array_equal(W.f32_to_e4m3_bits(mid + (hi - lo) * 1e-3), codes + 1)
+    np.testing.assert_array_equal(W.f32_to_e4m3_bits(-mid), even | 0x80)
+
+
+def test_fp8_cache_draws_and_poison():
+    s = W.WORKLOADS["gqa_fp8"].replace(batch=3, ctx=(5, 140))
+    x = W.make_inputs(s, seed=2, seq_lens=[5, 64, 140])
+    assert x["kv"].dtype == np.uint8 and x["kv"].shape == s.pool_shape(x["kv"].shape[0])
+    inside = []
+    for b, L in enumerate([5, 64, 140]):
+        for j in range(L):
+            page, slot = W.token_location(x, b, j)
+            inside.append(x["kv"][page, :, slot])
+    inside = np.concatenate([v.ravel() for v in inside])
+    assert not np.isin(inside, [0x7F, 0xFF]).any()           # no NaN inside any context
+    # slot 5 of the first sequence's page is past its context: poison codes only
+    page, _ = W.token_location(x, 0, 0)
+    assert np.isin(x["kv"][page, :, 5:], W.POISON_FP8).all()
+
+
 def test_deterministic_and_seeded():
     s = W.Shape("gqa", 3, 8, 2, 16, 0, (10, 200))
     a = W.make_inputs(s, seed=4)
