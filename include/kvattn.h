@@ -39,7 +39,9 @@
  *   kv_cache   latent variants: bf16 [num_pages][page_size][num_kv*d_nope + d_rope],
  *              each token row [c_0 | ... | c_{num_kv-1} | k_rope];
  *              GQA/MQA: bf16 [num_pages][2 (K, V)][page_size][num_kv][d_nope];
- *              GTA: bf16 [num_pages][page_size][num_kv][d_nope] (one tied plane)
+ *              GTA: bf16 [num_pages][page_size][num_kv][d_nope] (one tied plane);
+ *              GQA with cache_dtype FP8_E4M3: the GQA layout with one e4m3 byte
+ *              per element
  *   block_table int32 [B][max_pages_per_seq]: physical page of each logical
  *              64-token page; NULL = contiguous cache, sequence b owns pages
  *              b*max_pages_per_seq .. b*max_pages_per_seq + max_pages_per_seq-1
