@@ -620,7 +620,7 @@ def run_reference(args):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(full_s * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": describe(names), "name": args.workload, "batch_per_gpu": batch,
+        "config": {"workload": describe(names), "name": "+".join(names), "batch_per_gpu": batch,
                    "page_size": 64, "seed": args.seed},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.default_threads(),
                          "kind": "oracle", "sample": sample},
